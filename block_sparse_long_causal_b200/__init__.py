@@ -1,0 +1,188 @@
+"""Thin Python binding of libfp (FlashPrefill-style block-sparse causal prefill on sm_100a).
+
+Argument marshalling only: every step of the path (pooling, search, attention) runs in the
+CUDA kernels of libfp.so; PyTorch supplies device memory and the current stream. There is no
+CPU or PyTorch fallback: importing this module without the built library raises.
+
+Entry points mirror the C ABI in include/fp.h:
+    problem(...)            -> Problem (fp_problem_init)
+    block_pool(...)         -> fp_block_pool
+    block_search(...)       -> fp_block_search
+    block_sparse_attn(...)  -> fp_block_sparse_attn
+    dense_attn(...)         -> fp_dense_attn
+    validate_lists(...)     -> fp_validate_lists
+and SparsePrefill bundles the three steps with caller-side buffers.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp.so")
+
+FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 1, 2, 3, 4
+FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
+FP_MAX_SEQS = 1024
+EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_sparse_attn", "fp_dense_attn",
+            "fp_validate_lists", "fp_last_error", "fp_version")
+
+
+class FpError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"fp status {status}: {msg}")
+        self.status = status
+
+
+class fp_problem(C.Structure):
+    _fields_ = [("cu_seqlens", C.c_void_p), ("num_seqs", C.c_int32), ("total_tokens", C.c_int32),
+                ("total_blocks", C.c_int32), ("max_seq_blocks", C.c_int32), ("index_elems", C.c_int64),
+                ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
+                ("block_size", C.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libfp.so is not built ({LIB_PATH}); run python -m block_sparse_long_causal_b200.build")
+    lib = C.CDLL(LIB_PATH)
+    vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
+    P = C.POINTER(fp_problem)
+    sig = {
+        "fp_problem_init": [P, vp, i32, vp, i32, i32, i32, i32],
+        "fp_block_pool": [P, vp, vp, vp, vp, vp],
+        "fp_block_search": [P, vp, vp, f32, vp, vp, vp, vp],
+        "fp_block_sparse_attn": [P, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
+        "fp_dense_attn": [P, vp, vp, vp, f32, vp, vp, vp, vp],
+        "fp_validate_lists": [P, vp, vp, vp, vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = C.c_int
+    lib.fp_last_error.restype = C.c_char_p
+    lib.fp_last_error.argtypes = []
+    lib.fp_version.restype = C.c_int32
+    lib.fp_version.argtypes = []
+    return lib
+
+
+_lib = _load()
+
+
+def version() -> int:
+    return int(_lib.fp_version())
+
+
+def _check(st: int):
+    if st != FP_OK:
+        raise FpError(st, _lib.fp_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        return C.c_void_p(t.data_ptr())
+    return C.c_void_p(int(t))
+
+
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+class Problem:
+    """fp_problem plus the device cu_seqlens tensor it points to (kept alive here)."""
+
+    def __init__(self, cu_seqlens_host, cu_seqlens_dev: torch.Tensor, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, block_size: int):
+        host = np.ascontiguousarray(cu_seqlens_host, np.int32)
+        if cu_seqlens_dev.dtype != torch.int32:
+            raise ValueError("cu_seqlens must be int32")
+        self.cu_host = host
+        self.cu_dev = cu_seqlens_dev
+        self.c = fp_problem()
+        _check(_lib.fp_problem_init(C.byref(self.c), host.ctypes.data_as(C.c_void_p), len(host) - 1,
+                                    _ptr(cu_seqlens_dev), num_q_heads, num_kv_heads, head_dim, block_size))
+
+    def __getattr__(self, name):
+        return getattr(self.__dict__["c"], name)
+
+    @property
+    def ref(self):
+        return C.byref(self.c)
+
+
+def problem(cu_seqlens_host, num_q_heads: int, num_kv_heads: int, head_dim: int = 128, block_size: int = 128,
+            device="cuda") -> Problem:
+    host = np.ascontiguousarray(cu_seqlens_host, np.int32)
+    dev = torch.from_numpy(host.copy()).to(device)
+    return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size)
+
+
+def block_pool(p: Problem, q, k, q_pool, k_pool, stream=None):
+    _check(_lib.fp_block_pool(p.ref, _ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), _stream(stream)))
+
+
+def block_search(p: Problem, q_pool, k_pool, tau: float, counts, indices, dev_status=None, stream=None):
+    _check(_lib.fp_block_search(p.ref, _ptr(q_pool), _ptr(k_pool), float(tau), _ptr(counts), _ptr(indices),
+                                _ptr(dev_status), _stream(stream)))
+
+
+def block_sparse_attn(p: Problem, q, k, v, counts, indices, softmax_scale: float, out, lse=None, dev_status=None,
+                      stream=None):
+    _check(_lib.fp_block_sparse_attn(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(counts), _ptr(indices),
+                                     float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
+def dense_attn(p: Problem, q, k, v, softmax_scale: float, out, lse=None, dev_status=None, stream=None):
+    _check(_lib.fp_dense_attn(p.ref, _ptr(q), _ptr(k), _ptr(v), float(softmax_scale), _ptr(out), _ptr(lse),
+                              _ptr(dev_status), _stream(stream)))
+
+
+def validate_lists(p: Problem, counts, indices, dev_status, stream=None):
+    _check(_lib.fp_validate_lists(p.ref, _ptr(counts), _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
+class SparsePrefill:
+    """Caller-side buffers for one problem shape, and the three-step sparse prefill.
+
+    Buffers are allocated once (through PyTorch) and reused by every call; the library itself
+    never allocates.
+    """
+
+    def __init__(self, p: Problem, device="cuda", with_lse: bool = False):
+        self.p = p
+        nb, hq, hkv, d = p.total_blocks, p.num_q_heads, p.num_kv_heads, p.head_dim
+        self.q_pool = torch.empty((max(nb, 1), hq, d), dtype=torch.float32, device=device)
+        self.k_pool = torch.empty((max(nb, 1), hkv, d), dtype=torch.float32, device=device)
+        self.counts = torch.zeros((hq, max(nb, 1)), dtype=torch.int32, device=device)
+        self.indices = torch.zeros(max(p.index_elems, 1), dtype=torch.int32, device=device)
+        self.out = torch.empty((max(p.total_tokens, 1), hq, d), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((hq, max(p.total_tokens, 1)), dtype=torch.float32, device=device) if with_lse else None
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def search(self, q, k, tau: float, stream=None):
+        block_pool(self.p, q, k, self.q_pool, self.k_pool, stream)
+        block_search(self.p, self.q_pool, self.k_pool, tau, self.counts, self.indices, self.dev_status, stream)
+
+    def attend(self, q, k, v, softmax_scale: float = 0.0, stream=None):
+        block_sparse_attn(self.p, q, k, v, self.counts, self.indices, softmax_scale, self.out, self.lse,
+                          self.dev_status, stream)
+        return self.out
+
+    def __call__(self, q, k, v, tau: float, softmax_scale: float = 0.0, stream=None):
+        self.search(q, k, tau, stream)
+        return self.attend(q, k, v, softmax_scale, stream)
+
+    def dense(self, q, k, v, softmax_scale: float = 0.0, stream=None):
+        dense_attn(self.p, q, k, v, softmax_scale, self.out, self.lse, self.dev_status, stream)
+        return self.out

@@ -1,0 +1,270 @@
+// fp_api.cu -- the extern "C" boundary of libfp: argument checks, TMA tensor maps and launches.
+// See include/fp.h for the contract of every entry point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fp_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "no error";
+
+fp_status fail(fp_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+fp_status check_problem(const fp_problem* p) {
+  if (!p) return fail(FP_ERR_INVALID_ARG, "problem is NULL");
+  if (!p->cu_seqlens) return fail(FP_ERR_INVALID_ARG, "problem.cu_seqlens is NULL");
+  if (p->num_seqs < 1 || p->num_seqs > FP_MAX_SEQS)
+    return fail(FP_ERR_INVALID_ARG, "num_seqs=%d outside [1, %d]", p->num_seqs, FP_MAX_SEQS);
+  if (p->num_q_heads < 1 || p->num_kv_heads < 1 || p->num_q_heads % p->num_kv_heads)
+    return fail(FP_ERR_INVALID_ARG, "num_q_heads=%d must be a positive multiple of num_kv_heads=%d",
+                p->num_q_heads, p->num_kv_heads);
+  if (p->num_q_heads / p->num_kv_heads > 64)
+    return fail(FP_ERR_UNSUPPORTED, "GQA group size %d > 64", p->num_q_heads / p->num_kv_heads);
+  if (p->head_dim != 128) return fail(FP_ERR_UNSUPPORTED, "head_dim=%d (only 128 is built)", p->head_dim);
+  if (p->block_size != 64 && p->block_size != 128)
+    return fail(FP_ERR_UNSUPPORTED, "block_size=%d (64 or 128)", p->block_size);
+  if (p->total_tokens < 0 || p->total_blocks < 0 || p->index_elems < 0)
+    return fail(FP_ERR_INVALID_ARG, "negative sizes in problem (use fp_problem_init)");
+  return FP_OK;
+}
+
+fp::SeqInfo seq_info(const fp_problem* p) {
+  fp::SeqInfo s;
+  s.cu_seqlens = p->cu_seqlens;
+  s.num_seqs = p->num_seqs;
+  s.total_tokens = p->total_tokens;
+  s.total_blocks = p->total_blocks;
+  s.block = p->block_size;
+  return s;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 [rows, cols] row-major, box {64 cols, box_rows}, 128-byte swizzle, zero fill out of range.
+fp_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP_OK;
+}
+
+fp_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return FP_OK;
+  return fail(FP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* s = getenv("FP_WAIT_LIMIT_MS");
+    double ms = s ? atof(s) : 2000.0;
+    if (!(ms > 0.0)) ms = 2000.0;
+    return (uint64_t)(ms * 1e6);
+  }();
+  return v;
+}
+
+fp_status attn_common(const fp_problem* p, const void* q, const void* k, const void* v, const int32_t* counts,
+                      const int32_t* indices, int dense, float softmax_scale, void* out, float* lse,
+                      int32_t* dev_status, void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!q || !k || !v || !out) return fail(FP_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  if (!dense && (!counts || !indices)) return fail(FP_ERR_INVALID_ARG, "counts and indices must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(FP_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(FP_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if (p->total_tokens == 0) return FP_OK;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)p->head_dim);
+
+  fp::AttnParams a;
+  memset(&a, 0, sizeof a);
+  const int64_t T = p->total_tokens;
+  if ((st = make_tmap(&a.tm_q, q, T, (int64_t)p->num_q_heads * p->head_dim, fp::kTileM)) != FP_OK) return st;
+  if ((st = make_tmap(&a.tm_k, k, T, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
+  if ((st = make_tmap(&a.tm_v, v, T, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
+  a.seq = seq_info(p);
+  a.hq = p->num_q_heads;
+  a.hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  // exact tile count comes from the device tables; the grid uses an upper bound
+  const long long tiles_ub = (long long)p->num_q_heads * ((T + fp::kTileM - 1) / fp::kTileM + p->num_seqs);
+  a.num_tiles = 0;
+  a.dense = dense;
+  a.counts = counts;
+  a.indices = indices;
+  a.index_elems = p->index_elems;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.dev_status = dev_status;
+  a.wait_limit_ns = wait_limit_ns();
+  const int grid = (int)(tiles_ub < sm_count() ? tiles_ub : sm_count());
+  return cuda_status(fp::launch_attn(a, grid, static_cast<cudaStream_t>(stream)), "attention launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+fp_status fp_problem_init(fp_problem* p, const int32_t* host_cu, int32_t num_seqs, const int32_t* dev_cu,
+                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size) {
+  if (!p || !host_cu || !dev_cu) return fail(FP_ERR_INVALID_ARG, "NULL argument to fp_problem_init");
+  if (num_seqs < 1 || num_seqs > FP_MAX_SEQS)
+    return fail(FP_ERR_INVALID_ARG, "num_seqs=%d outside [1, %d]", num_seqs, FP_MAX_SEQS);
+  if (block_size != 64 && block_size != 128)
+    return fail(FP_ERR_UNSUPPORTED, "block_size=%d (64 or 128)", block_size);
+  if (host_cu[0] != 0) return fail(FP_ERR_INVALID_ARG, "cu_seqlens[0] must be 0");
+  int64_t nb_tot = 0, idx = 0, max_nb = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int64_t L = (int64_t)host_cu[s + 1] - host_cu[s];
+    if (L < 0) return fail(FP_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing (sequence %d)", s);
+    const int64_t nb = (L + block_size - 1) / block_size;
+    nb_tot += nb;
+    idx += (int64_t)num_q_heads * nb * (nb + 1) / 2;
+    if (nb > max_nb) max_nb = nb;
+  }
+  if (host_cu[num_seqs] > (int64_t)INT32_MAX / 2 || nb_tot > INT32_MAX)
+    return fail(FP_ERR_INVALID_ARG, "too many tokens");
+  memset(p, 0, sizeof *p);
+  p->cu_seqlens = dev_cu;
+  p->num_seqs = num_seqs;
+  p->total_tokens = host_cu[num_seqs];
+  p->total_blocks = (int32_t)nb_tot;
+  p->max_seq_blocks = (int32_t)max_nb;
+  p->index_elems = idx;
+  p->num_q_heads = num_q_heads;
+  p->num_kv_heads = num_kv_heads;
+  p->head_dim = head_dim;
+  p->block_size = block_size;
+  return check_problem(p);
+}
+
+fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float* q_pool, float* k_pool,
+                        void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "q, k, q_pool and k_pool must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool))
+    return fail(FP_ERR_INVALID_ARG, "q, k, q_pool and k_pool must be 16-byte aligned");
+  if (p->total_blocks == 0) return FP_OK;
+  fp::PoolParams a;
+  a.seq = seq_info(p);
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.q_pool = q_pool;
+  a.k_pool = k_pool;
+  a.q_row = p->num_q_heads * p->head_dim;
+  a.k_row = p->num_kv_heads * p->head_dim;
+  a.q_chunks = (a.q_row + 1023) / 1024;
+  a.k_chunks = (a.k_row + 1023) / 1024;
+  a.dev_status = nullptr;
+  const long long items = (long long)p->total_blocks * (a.q_chunks + a.k_chunks);
+  const long long cap = (long long)sm_count() * 16;
+  const int grid = (int)(items < cap ? items : cap);
+  return cuda_status(fp::launch_pool(a, grid, static_cast<cudaStream_t>(stream)), "pool launch");
+}
+
+fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
+                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!q_pool || !k_pool || !counts || !indices)
+    return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, counts and indices must be non-NULL");
+  if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
+  if (!std::isfinite(tau)) return fail(FP_ERR_INVALID_ARG, "tau must be finite");
+  if (p->total_blocks == 0) return FP_OK;
+  fp::SearchParams a;
+  a.seq = seq_info(p);
+  a.q_pool = q_pool;
+  a.k_pool = k_pool;
+  a.hq = p->num_q_heads;
+  a.hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.rows_blocks = 64 / a.group > 0 ? 64 / a.group : 1;
+  // tiles = Hkv * sum_s ceil(nb_s / TI), counted on the device; the grid uses an upper bound
+  a.num_tiles = (int32_t)((long long)p->num_kv_heads * (p->total_blocks / a.rows_blocks + p->num_seqs));
+  a.inv_sqrt_d = 1.0f / std::sqrt((float)p->head_dim);
+  a.keep_all = tau <= 0.f;
+  a.log_tau = tau > 0.f ? (float)std::log((double)tau) : -INFINITY;
+  a.counts = counts;
+  a.indices = indices;
+  a.index_elems = p->index_elems;
+  a.dev_status = dev_status;
+  return cuda_status(fp::launch_search(a, static_cast<cudaStream_t>(stream)), "search launch");
+}
+
+fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,
+                               const int32_t* counts, const int32_t* indices, float softmax_scale, void* out,
+                               float* lse, int32_t* dev_status, void* stream) {
+  return attn_common(p, q, k, v, counts, indices, 0, softmax_scale, out, lse, dev_status, stream);
+}
+
+fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
+                        void* out, float* lse, int32_t* dev_status, void* stream) {
+  return attn_common(p, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
+}
+
+fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices, int32_t* dev_status,
+                            void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!counts || !indices || !dev_status)
+    return fail(FP_ERR_INVALID_ARG, "counts, indices and dev_status must be non-NULL");
+  if (p->total_blocks == 0) return FP_OK;
+  fp::ValidateParams a;
+  a.seq = seq_info(p);
+  a.hq = p->num_q_heads;
+  a.counts = counts;
+  a.indices = indices;
+  a.index_elems = p->index_elems;
+  a.dev_status = dev_status;
+  return cuda_status(fp::launch_validate(a, static_cast<cudaStream_t>(stream)), "validate launch");
+}
+
+const char* fp_last_error(void) { return g_err; }
+
+int32_t fp_version(void) { return 100; }
+
+}  // extern "C"

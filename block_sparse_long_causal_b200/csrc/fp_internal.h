@@ -1,0 +1,84 @@
+// fp_internal.h -- launch parameter structs and launcher declarations shared by the CUDA sources
+// of libfp (not part of the public ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/fp.h"
+
+namespace fp {
+
+struct SeqInfo {
+  const int32_t* cu_seqlens;  // device [S+1]
+  int32_t num_seqs;
+  int32_t total_tokens;
+  int32_t total_blocks;
+  int32_t block;              // B
+};
+
+struct PoolParams {
+  SeqInfo seq;
+  const uint16_t* q;          // [T, Hq, d] bf16 bits
+  const uint16_t* k;          // [T, Hkv, d]
+  float* q_pool;              // [NB, Hq, d]
+  float* k_pool;              // [NB, Hkv, d]
+  int32_t q_row;              // Hq * d
+  int32_t k_row;              // Hkv * d
+  int32_t q_chunks, k_chunks; // 1024-element column chunks per token row
+  int32_t* dev_status;
+};
+
+struct SearchParams {
+  SeqInfo seq;
+  const float* q_pool;
+  const float* k_pool;
+  int32_t hq, hkv, group;     // group = Hq / Hkv
+  int32_t rows_blocks;        // query blocks per CTA tile (TI)
+  int32_t num_tiles;          // grid-size hint (upper bound); the exact count is s_ct[S] on device
+  float inv_sqrt_d;
+  float log_tau;              // threshold on s - max (natural log units); -inf keeps all
+  int32_t keep_all;           // tau <= 0
+  int32_t* counts;            // [Hq, NB]
+  int32_t* indices;           // triangular
+  int64_t index_elems;
+  int32_t* dev_status;
+};
+
+struct ValidateParams {
+  SeqInfo seq;
+  int32_t hq;
+  const int32_t* counts;
+  const int32_t* indices;
+  int64_t index_elems;
+  int32_t* dev_status;
+};
+
+struct __align__(64) AttnParams {
+  CUtensorMap tm_q;           // Q as 2-D [T rows, Hq*d cols], box {64, 128}, 128B swizzle
+  CUtensorMap tm_k;           // K as 2-D [T rows, Hkv*d cols], box {64, B}
+  CUtensorMap tm_v;           // V likewise
+  SeqInfo seq;
+  int32_t hq, hkv, group;
+  int32_t num_tiles;          // unused by the kernel (exact count is s_ct[S] on device)
+  int32_t dense;              // 1: every causal block; 0: counts/indices lists
+  const int32_t* counts;
+  const int32_t* indices;
+  int64_t index_elems;
+  float scale_log2;           // softmax_scale * log2(e)
+  uint16_t* out;              // [T, Hq, d] bf16 bits
+  float* lse;                 // [Hq, T] or null
+  int32_t* dev_status;
+  uint64_t wait_limit_ns;
+};
+
+constexpr int kMaxSeqs = FP_MAX_SEQS;
+constexpr int kHeadDim = 128;
+constexpr int kTileM = 128;   // query rows per attention tile
+
+cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st);
+cudaError_t launch_search(const SearchParams& p, cudaStream_t st);
+cudaError_t launch_validate(const ValidateParams& p, cudaStream_t st);
+cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st);
+
+}  // namespace fp

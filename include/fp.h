@@ -1,0 +1,139 @@
+/*
+ * fp.h -- C ABI of the B200 (sm_100a) FlashPrefill-style block-sparse causal prefill library
+ *         (libfp.so).
+ *
+ * The method (FlashPrefill, "Instantaneous Pattern Discovery and Thresholding for Ultra-Fast
+ * Long-Context Prefilling"):
+ *   1. pool     mean-pool Q and K over B-token blocks (skill summary page, "Stage 1: Block-Level
+ *               Attention Approximation"; "Architecture Overview": "average-pooled keys/queries");
+ *   2. search   pooled block scores s_ij = qbar_i . kbar_j / sqrt(d) (same section), causal softmax
+ *               p_ij over j <= i, keep block j iff p_ij >= tau * max_j p_ij ("Core Concept" item 3,
+ *               "Dynamic Thresholding": one max reduction, no sorting or cumulative sums); the sink
+ *               block 0 and the diagonal block i are always kept; kept blocks are written as
+ *               ascending per-(head, query block) index lists ("Physical Index Jumping");
+ *   3. attend   block-sparse causal flash attention over exactly the listed blocks, online softmax
+ *               (FlashPrefill V2 abstract: block-sparse prefill attention operator).
+ * A dense causal kernel built the same way is the baseline (FlashPrefill V2 abstract: "dense
+ * baseline").
+ *
+ * Conventions shared by every call
+ *   - Tensors are row-major [tokens, heads, head_dim]; Q has num_q_heads heads, K and V have
+ *     num_kv_heads heads; q-head h reads kv-head h / (num_q_heads / num_kv_heads) (GQA).
+ *     Q, K, V and O hold bf16 bit patterns (2 bytes per element).
+ *   - Several sequences may be packed along tokens (varlen): device cu_seqlens[s]..cu_seqlens[s+1]
+ *     is sequence s. Each sequence is causal on its own (query position == key position space, no
+ *     cached prefix); blocks, the sink block and block ids restart at every sequence.
+ *   - Block b of a sequence of length L spans local tokens [b*B, min((b+1)*B, L)); nb = ceil(L/B).
+ *     Global block id of (sequence s, local block i) = sum_{s'<s} nb_{s'} + i.
+ *   - Pooled tensors: float32 [total_blocks, heads, head_dim].
+ *   - counts: int32 [num_q_heads, total_blocks]: number of kept blocks of row (h, global block).
+ *   - indices: int32, triangular-packed: row (s, h, i) starts at
+ *         base_s + h * nb_s*(nb_s+1)/2 + i*(i+1)/2,   base_s = sum_{s'<s} Hq * nb_{s'}(nb_{s'}+1)/2,
+ *     has room for i+1 entries, and holds the kept LOCAL block ids in ascending order.
+ *     fp_problem.index_elems is the buffer length in int32 elements.
+ *   - The caller owns every buffer. The library never allocates or frees device memory and never
+ *     synchronises: every call only enqueues kernels on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream). Pointers marked "device" must be device-accessible and 16-byte
+ *     aligned.
+ *   - Host-side checks run before any launch; a non-OK status means nothing was enqueued, and
+ *     fp_last_error() describes the problem. FP_ERR_CUDA means a launch failed.
+ *   - dev_status (optional, device int32, may be NULL): kernels OR FP_DEV_* bits into it when a
+ *     bounded wait gives up or an index entry is out of range (the entry is skipped). Read it
+ *     after the stream has completed. Kernels never trap.
+ */
+#ifndef FP_H_
+#define FP_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP_API __attribute__((visibility("default")))
+#else
+#define FP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp_status {
+  FP_OK = 0,
+  FP_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer, non-finite tau, ... */
+  FP_ERR_UNSUPPORTED = 2,  /* valid but not implemented here (head_dim != 128, B not 64/128) */
+  FP_ERR_CUDA = 3,         /* a CUDA launch or driver call failed */
+  FP_ERR_TIMEOUT = 4       /* reserved for callers that map FP_DEV_TIMEOUT to a status */
+} fp_status;
+
+/* Bits written into dev_status by the kernels. */
+#define FP_DEV_TIMEOUT 1     /* a bounded mbarrier wait gave up; outputs of that launch are undefined */
+#define FP_DEV_BAD_LIST 2    /* an index-list entry or count was out of range and was skipped/clamped */
+#define FP_DEV_BAD_PROBLEM 4 /* device cu_seqlens disagree with the sizes in fp_problem */
+
+#define FP_MAX_SEQS 1024     /* maximum number of packed sequences per call */
+
+/* Shared description of one prefill problem. Fill it with fp_problem_init. */
+typedef struct fp_problem {
+  const int32_t* cu_seqlens; /* device, [num_seqs+1], cu_seqlens[0] = 0, non-decreasing */
+  int32_t num_seqs;          /* 1 .. FP_MAX_SEQS */
+  int32_t total_tokens;      /* cu_seqlens[num_seqs] */
+  int32_t total_blocks;      /* sum_s ceil(L_s / B) */
+  int32_t max_seq_blocks;    /* max_s ceil(L_s / B) */
+  int64_t index_elems;       /* int32 entries of the triangular index buffer */
+  int32_t num_q_heads;       /* Hq, a multiple of num_kv_heads */
+  int32_t num_kv_heads;      /* Hkv */
+  int32_t head_dim;          /* d; 128 is supported */
+  int32_t block_size;        /* B; 64 or 128 */
+} fp_problem;
+
+/* Fill *p from a HOST copy of cu_seqlens (read only during the call) and the device copy that the
+ * kernels will read. Checks sizes and the sequence limits. */
+FP_API fp_status fp_problem_init(fp_problem* p, const int32_t* host_cu_seqlens, int32_t num_seqs,
+                          const int32_t* dev_cu_seqlens, int32_t num_q_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t block_size);
+
+/* Step 1 -- block mean pooling (FlashPrefill skill summary page, "Stage 1").
+ * q: device bf16 [total_tokens, Hq, d]; k: device bf16 [total_tokens, Hkv, d].
+ * q_pool: device float32 [total_blocks, Hq, d]; k_pool: device float32 [total_blocks, Hkv, d].
+ * The mean of a partial last block is over the tokens it holds. */
+FP_API fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float* q_pool, float* k_pool,
+                        void* stream);
+
+/* Step 2 -- pooled block scores, causal softmax, max-based threshold, index emission
+ * (FlashPrefill skill summary page, "Stage 1" and "Core Concept" item 3; "Physical Index Jumping").
+ * Keeps block j of row (h, i) iff exp(s_ij - max_j s_ij) >= tau (equal to p_ij >= tau * max_j p_ij),
+ * plus j = 0 and j = i. tau <= 0 keeps every causal block; tau must be finite.
+ * q_pool/k_pool: outputs of fp_block_pool. counts: device int32 [Hq, total_blocks];
+ * indices: device int32 [index_elems] (entries past a row's count are left untouched). */
+FP_API fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
+                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream);
+
+/* Step 3 -- block-sparse causal attention over the listed blocks (online softmax, bf16 in,
+ * fp32 accumulate, bf16 out). counts/indices as written by fp_block_search (any ascending lists
+ * of local block ids <= i are accepted; out-of-range entries are skipped and flagged).
+ * softmax_scale <= 0 selects 1/sqrt(d). out: device bf16 [total_tokens, Hq, d].
+ * lse (optional, may be NULL): device float32 [Hq, total_tokens], natural-log sum of
+ * exp(softmax_scale * q.k) over the attended keys. */
+FP_API fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,
+                               const int32_t* counts, const int32_t* indices, float softmax_scale, void* out,
+                               float* lse, int32_t* dev_status, void* stream);
+
+/* Dense causal attention (every causal block), same kernel design; the baseline for the speedup. */
+FP_API fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
+                        void* out, float* lse, int32_t* dev_status, void* stream);
+
+/* Device-side check of index lists: every row's count in [1, i+1], entries ascending, in [0, i],
+ * first entry 0 and last entry i. Violations OR FP_DEV_BAD_LIST into dev_status (required). */
+FP_API fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices,
+                            int32_t* dev_status, void* stream);
+
+/* Message for the last non-OK status returned on this thread (never NULL). */
+FP_API const char* fp_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+FP_API int32_t fp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP_H_ */

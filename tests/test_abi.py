@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every entry point declared in include/fp.h, and rejects bad
+arguments on the host before any launch (no GPU needed for any of these)."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_long_causal_b200 as fp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "fp.h")) as f:
+        return sorted(set(re.findall(r"FP_API\s+[\w\s\*]+?\b(fp_\w+)\s*\(", f.read())))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("fp_block_pool", "fp_block_search", "fp_block_sparse_attn", "fp_dense_attn"):
+        assert n in names
+    assert set(names) == set(fp.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(fp.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert fp.version() >= 100
+
+
+def _prob(cu=(0, 300), hq=4, hkv=2, d=128, B=128):
+    p = fp.fp_problem()
+    host = np.array(cu, np.int32)
+    st = fp._lib.fp_problem_init(C.byref(p), host.ctypes.data_as(C.c_void_p), len(host) - 1, C.c_void_p(16),
+                                 hq, hkv, d, B)
+    return st, p
+
+
+def _err():
+    return fp._lib.fp_last_error().decode()
+
+
+def test_problem_init_sizes():
+    st, p = _prob((0, 300, 301, 700), hq=3, hkv=1, B=64)
+    assert st == fp.FP_OK
+    assert p.total_tokens == 700 and p.total_blocks == 5 + 1 + 7 and p.max_seq_blocks == 7
+    assert p.index_elems == 3 * (15 + 1 + 28)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), fp.FP_ERR_UNSUPPORTED),
+    (dict(B=32), fp.FP_ERR_UNSUPPORTED),
+    (dict(hq=6, hkv=4), fp.FP_ERR_INVALID_ARG),
+    (dict(hq=0, hkv=1), fp.FP_ERR_INVALID_ARG),
+    (dict(cu=(1, 5)), fp.FP_ERR_INVALID_ARG),
+    (dict(cu=(0, 9, 5)), fp.FP_ERR_INVALID_ARG),
+    (dict(hq=128, hkv=1), fp.FP_ERR_UNSUPPORTED),
+])
+def test_problem_init_rejects(kw, status):
+    st, _ = _prob(**kw)
+    assert st == status, _err()
+    assert _err()
+
+
+def test_problem_init_rejects_too_many_sequences():
+    st, _ = _prob(cu=tuple(range(fp.FP_MAX_SEQS + 2)))
+    assert st == fp.FP_ERR_INVALID_ARG
+
+
+def test_empty_sequences_are_allowed():
+    st, p = _prob(cu=(0, 0, 5, 5))
+    assert st == fp.FP_OK and p.total_blocks == 1
+
+
+def test_calls_reject_bad_arguments_before_launch():
+    st, p = _prob()
+    assert st == fp.FP_OK
+    ok = C.c_void_p(4096)
+    mis = C.c_void_p(4098)
+    null = None
+    pr = C.byref(p)
+    s = None
+    assert fp._lib.fp_block_pool(pr, null, ok, ok, ok, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_pool(pr, mis, ok, ok, ok, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_search(pr, ok, ok, C.c_float(float("nan")), ok, ok, null, s) == fp.FP_ERR_INVALID_ARG
+    assert "tau" in _err()
+    assert fp._lib.fp_block_search(pr, ok, ok, C.c_float(float("inf")), ok, ok, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_search(pr, ok, null, C.c_float(0.1), ok, ok, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_sparse_attn(pr, ok, ok, ok, null, ok, C.c_float(0), ok, null, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_sparse_attn(pr, ok, ok, mis, ok, ok, C.c_float(0), ok, null, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_dense_attn(pr, ok, ok, ok, C.c_float(float("nan")), ok, null, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_dense_attn(None, ok, ok, ok, C.c_float(0), ok, null, null, s) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_validate_lists(pr, ok, ok, null, s) == fp.FP_ERR_INVALID_ARG
+    # a problem edited into an unsupported state is rejected by every call
+    p.head_dim = 96
+    assert fp._lib.fp_dense_attn(pr, ok, ok, ok, C.c_float(0), ok, null, null, s) == fp.FP_ERR_UNSUPPORTED
+
+
+def test_binding_raises_fp_error():
+    with pytest.raises(fp.FpError):
+        fp.Problem(np.array([0, 10], np.int32), __import__("torch").zeros(2, dtype=__import__("torch").int32),
+                   4, 2, 64, 128)

@@ -1,0 +1,93 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Index lists: bit-exact outside the tie band (|p/max p - tau| <= 1e-4 tau).
+Attention: oracle on the GPU's own lists; max-abs <= 2e-2, mean-abs <= 2e-3 (bf16 I/O, fp32
+accumulation), plus a relative L2 error bound of 2e-2 so that real bugs are not hidden by the small
+magnitude of long-context outputs.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from helpers import compare_attention, compare_lists, gpu_prefill, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import block_sparse_long_causal_b200  # noqa: F401  (fails loudly without libfp.so)
+
+
+def _oracle_lists(x, B, tau):
+    cu = x["cu_seqlens"]
+    qb, kb = oracle.pool(x["q"], cu, B), oracle.pool(x["k"], cu, B)
+    return qb, kb, oracle.search(qb, kb, cu, B, tau)
+
+
+def _check_case(x, hq, hkv, B, tau, rows=None, rel_max=2e-2):
+    res = gpu_prefill(x, hq, hkv, B, tau)
+    qb, kb, (oc, oi, band) = _oracle_lists(x, B, tau)
+    np.testing.assert_allclose(res["q_pool"], qb, rtol=0, atol=5e-5)
+    np.testing.assert_allclose(res["k_pool"], kb, rtol=0, atol=5e-5)
+    nband, nkept = compare_lists(res["counts"], res["indices"], oc, oi, band, x["cu_seqlens"], B, hq)
+    if rows is None:
+        st = compare_attention(x, res, hq, B)
+    else:
+        st = compare_attention(x, res, hq, B, *rows)
+    assert st["rel"] <= rel_max, st
+    return res, st, nkept
+
+
+SMALL = [
+    # (lens, hq, hkv, B, tau, scale)
+    ((128,), 1, 1, 128, 0.1, 1.0),
+    ((300,), 2, 1, 128, 0.5, 3.0),
+    ((1,), 1, 1, 128, 0.1, 1.0),
+    ((1000,), 4, 2, 128, 0.9, 3.0),
+    ((257, 1, 130, 640), 8, 2, 128, 0.7, 3.0),
+    ((513,), 4, 4, 64, 0.5, 3.0),
+    ((64, 65, 127, 191), 4, 1, 64, 0.8, 3.0),
+    ((2048,), 8, 1, 128, 0.0, 1.0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"L{'-'.join(map(str, c[0]))}_h{c[1]}x{c[2]}_B{c[3]}_t{c[4]}")
+def test_small_ragged_cases(case):
+    lens, hq, hkv, B, tau, scale = case
+    x = synth.random_inputs(lens, hq, hkv, 128, seed=sum(lens) + hq, scale=scale)
+    _check_case(x, hq, hkv, B, tau)
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.95, 0.98])
+def test_mha4_L2048_B64(tau):
+    w = synth.WORKLOADS["mha4-L2048-B64"]
+    x = synth.make_inputs(w)
+    _check_case(x, w.hq, w.hkv, w.block, tau)
+
+
+def test_dense_matches_oracle_dense():
+    w = synth.WORKLOADS["mha4-L2048-B64"]
+    x = synth.make_inputs(w.with_lens([1500]))
+    res = gpu_prefill(x, w.hq, w.hkv, w.block, w.tau, dense=True)
+    st = compare_attention(x, res, w.hq, w.block, lists=False)
+    assert st["rel"] <= 2e-2
+
+
+def test_dense_equals_sparse_at_tau0_bitwise():
+    w = synth.WORKLOADS["llama3-8b-L32768"]
+    x = synth.make_inputs(w.with_lens([3000, 700]))
+    a = gpu_prefill(x, w.hq, w.hkv, w.block, 0.0, dense=False)
+    b = gpu_prefill(x, w.hq, w.hkv, w.block, 0.0, dense=True)
+    np.testing.assert_array_equal(a["out"], b["out"])
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.95])
+def test_llama3_8b_L32768(tau):
+    w = synth.WORKLOADS["llama3-8b-L32768"]
+    x = synth.make_inputs(w)
+    rows = sample_rows(x["cu_seqlens"], w.hq, 192, seed=1)
+    _check_case(x, w.hq, w.hkv, w.block, tau, rows=rows)
