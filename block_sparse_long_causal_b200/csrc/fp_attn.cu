@@ -29,6 +29,7 @@
 namespace fp {
 
 constexpr int kThreads = 192;
+constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0, kTmemO = 256;
 
@@ -357,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       int j, mask, n = 0;
       while (itr.next(j, mask)) {
         const uint32_t b = it & 1;
-        if (!mbar_wait(b_s_full0 + 8 * b, (it >> 1) & 1, p.wait_limit_ns)) { fail = true; break; }
+        // tcgen05.ld/st are warp-collective: every branch around them is made warp-uniform
+        if (__any_sync(kFull, !mbar_wait(b_s_full0 + 8 * b, (it >> 1) & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
         uint32_t sr[BK];
 #pragma unroll
@@ -376,24 +378,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         const float m_tile = mx * p.scale_log2;
         const float m_new = fmaxf(m_run, m_tile);
-        if (m_new > m_run + 8.0f) {           // grow the reference max (lazy rescale)
-          const float alpha = ex2_approx(m_run - m_new);
-          if (n > 0) {
-            // O must hold PV_{n-1} before it is rescaled
-            if (!mbar_wait(b_o_done, (it - 1) & 1, p.wait_limit_ns)) { fail = true; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kHeadDim; c += 32) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_off + kTmemO + c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tmem + lane_off + kTmemO + c, o);
-            }
-          }
-          l_run *= alpha;
+        // grow the reference max only when it rises by more than 2^8 (lazy rescale); the stale
+        // max is exact because the numerator and the denominator share it
+        const bool grow = m_new > m_run + 8.0f;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = ex2_approx(m_run - m_new);
           m_run = m_new;
+        }
+        l_run *= alpha;
+        if (n > 0 && __any_sync(kFull, grow)) {
+          // O must hold PV_{n-1} before it is rescaled (lanes that did not grow scale by 1)
+          if (__any_sync(kFull, !mbar_wait(b_o_done, (it - 1) & 1, p.wait_limit_ns))) { fail = true; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < kHeadDim; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + kTmemO + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tmem + lane_off + kTmemO + c, o);
+          }
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         float sum = 0.f;
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         ++n;
       }
       bad_list |= itr.bad;
-      if (fail || *s_abort) { fail = true; break; }
+      if (__any_sync(kFull, fail || *s_abort)) { fail = true; break; }
       const bool row_ok = qpos < tl.len;
       if (n == 0) {  // empty kv list (malformed input): zero output, LSE -inf
         if (row_ok) {
@@ -427,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         continue;
       }
       // ---- epilogue: O / l -> bf16, LSE
-      if (!mbar_wait(b_o_final, fc & 1, p.wait_limit_ns)) { fail = true; break; }
+      if (__any_sync(kFull, !mbar_wait(b_o_final, fc & 1, p.wait_limit_ns))) { fail = true; break; }
       ++fc;
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
