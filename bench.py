@@ -127,6 +127,15 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.rows)}
 
 
+def workload(args):
+    w = synth.WORKLOADS[args.workload]
+    if args.lens:
+        lens = [int(v) for v in args.lens.split(",")]
+        w = w.with_lens(lens, seeds=list(w.seeds[: len(lens)]) + list(range(len(w.seeds), len(lens))),
+                        name=f"{w.name}@lens={args.lens}")
+    return w
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
@@ -146,7 +155,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
 
-    w = synth.WORKLOADS[args.workload]
+    w = workload(args)
     tau = w.tau if args.tau is None else args.tau
     if ws > 1:  # independent replica per rank: distinct seeds
         w = w.with_lens(w.lens, seeds=[s + 1000 * rank for s in w.seeds])
@@ -386,7 +395,7 @@ def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    w = synth.WORKLOADS[args.workload]
+    w = workload(args)
     tau = w.tau if args.tau is None else args.tau
     x = synth.make_inputs(w)
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
@@ -420,6 +429,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--lens", type=str, default=None,
+                    help="comma-separated sequence lengths replacing the workload's (smaller case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -28,7 +28,7 @@ FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 
 FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
 FP_MAX_SEQS = 1024
 EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_sparse_attn", "fp_dense_attn",
-            "fp_validate_lists", "fp_last_error", "fp_version")
+            "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version")
 
 
 class FpError(RuntimeError):
@@ -46,7 +46,7 @@ class fp_problem(C.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libfp.so is not built ({LIB_PATH}); run python -m block_sparse_long_causal_b200.build")
+        raise ImportError(f"libfp.so is not built ({LIB_PATH}); run python block_sparse_long_causal_b200/build.py")
     lib = C.CDLL(LIB_PATH)
     vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
     P = C.POINTER(fp_problem)
@@ -57,6 +57,7 @@ def _load():
         "fp_block_sparse_attn": [P, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_dense_attn": [P, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_validate_lists": [P, vp, vp, vp, vp],
+        "fp_selftest_exp2": [vp, vp, vp, C.c_int64, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +151,10 @@ def dense_attn(p: Problem, q, k, v, softmax_scale: float, out, lse=None, dev_sta
 
 def validate_lists(p: Problem, counts, indices, dev_status, stream=None):
     _check(_lib.fp_validate_lists(p.ref, _ptr(counts), _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
+def selftest_exp2(x, y_poly, y_mufu, stream=None):
+    _check(_lib.fp_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(), _stream(stream)))
 
 
 class SparsePrefill:

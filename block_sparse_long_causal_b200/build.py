@@ -1,8 +1,9 @@
 """Build libfp.so (the sm_100a C-ABI library) in-tree with nvcc.
 
-    python -m block_sparse_long_causal_b200.build [--force] [--verbose]
+    python block_sparse_long_causal_b200/build.py [--force] [--verbose]
 
-The library is written next to this file so that it travels with the repository snapshot.
+The library is written next to this file so that it travels with the repository snapshot. Run it
+by path (not with -m): importing the package loads the library, which may not exist yet.
 """
 from __future__ import annotations
 

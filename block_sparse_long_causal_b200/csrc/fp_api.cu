@@ -263,6 +263,13 @@ fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const in
   return cuda_status(fp::launch_validate(a, static_cast<cudaStream_t>(stream)), "validate launch");
 }
 
+fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu)))
+    return fail(FP_ERR_INVALID_ARG, "x, y_poly and y_mufu must be non-NULL for n > 0");
+  return cuda_status(fp::launch_exp2_selftest(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)),
+                     "exp2 self-test launch");
+}
+
 const char* fp_last_error(void) { return g_err; }
 
 int32_t fp_version(void) { return 100; }

@@ -30,6 +30,8 @@ namespace fp {
 
 constexpr int kThreads = 192;
 constexpr unsigned kFull = 0xffffffffu;
+// exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU: 3 of 8
+constexpr unsigned kPolyPairs = 0xA4u;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0, kTmemO = 256;
 
@@ -368,13 +370,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         tmem_wait_ld();
         // causal mask (diagonal tiles) and the per-half list mask (B = 64)
         const int valid = ((mask >> (kTileM / BK == 2 ? half : 0)) & 1) ? (qpos - j * BK) : -1;
-        float mx = -INFINITY;
+        const bool masked = valid < BK - 1;   // this row needs element masking on this tile
+        float mx;
+        if (masked) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < BK; ++c) {
-          float v = __uint_as_float(sr[c]);
-          v = (c <= valid) ? v : -INFINITY;
-          sr[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int c = 0; c < BK; ++c) {
+            const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
+            sr[c] = __float_as_uint(v);
+            m4[c & 3] = fmaxf(m4[c & 3], v);
+          }
+          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        } else {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < BK; c += 8) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
+          }
+          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         }
         const float m_tile = mx * p.scale_log2;
         const float m_new = fmaxf(m_run, m_tile);
@@ -391,27 +406,63 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           // O must hold PV_{n-1} before it is rescaled (lanes that did not grow scale by 1)
           if (__any_sync(kFull, !mbar_wait(b_o_done, (it - 1) & 1, p.wait_limit_ns))) { fail = true; break; }
           tc_fence_after();
+          const uint64_t a2 = f2_make(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < kHeadDim; c += 32) {
             uint32_t o[32];
             tmem_ld32(tmem + lane_off + kTmemO + c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              float lo, hi;
+              f2_split(fmul2(f2_bits(o[e], o[e + 1]), a2), lo, hi);
+              o[e] = __float_as_uint(lo);
+              o[e + 1] = __float_as_uint(hi);
+            }
             tmem_st32(tmem + lane_off + kTmemO + c, o);
           }
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float sum = 0.f;
+        const uint64_t scale2 = f2_make(p.scale_log2, p.scale_log2);
+        const uint64_t negm2 = f2_make(-m_use, -m_use);
+        uint64_t sum2[2] = {0ull, 0ull};
         uint32_t pk[BK / 2];
+        if (masked) {
+          // exact zeros for masked keys: MUFU ex2(-inf) = 0
 #pragma unroll
-        for (int c = 0; c < BK; c += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), p.scale_log2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), p.scale_log2, -m_use));
-          sum += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < BK; c += 2) {
+            float x0, x1;
+            f2_split(ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2), x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2_make(p0, p1));
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // split exp2 between MUFU and the FMA-pipe polynomial (pairs whose index has a bit in
+          // kPolyPairs use the polynomial) so that neither unit alone bounds the softmax
+#pragma unroll
+          for (int c = 0; c < BK; c += 2) {
+            const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
+            uint64_t p2;
+            if ((kPolyPairs >> ((c >> 1) & 7)) & 1) {
+              p2 = exp2_poly2(x2);
+            } else {
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+            }
+            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
+            float p0, p1;
+            f2_split(p2, p0, p1);
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
         }
-        l_run += sum;
+        {
+          float a0, a1, b0, b1;
+          f2_split(sum2[0], a0, a1);
+          f2_split(sum2[1], b0, b1);
+          l_run += (a0 + a1) + (b0 + b1);
+        }
 #pragma unroll
         for (int c = 0; c < BK / 2; c += 32)
           tmem_st32(tmem + lane_off + kTmemS + 128 * b + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));

@@ -173,6 +173,74 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ---- packed fp32x2 arithmetic (sm_100a): one instruction, two lanes of a 64-bit register pair
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_bits(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe, for x <= 2^22 (inputs below -126 are clamped to -126).
+// Range reduction x = n + f with n = round-to-nearest(x) taken from the low mantissa bits of
+// x + 1.5*2^23 and f in [-0.5, 0.5]; 2^f by a degree-3 polynomial whose coefficients are a
+// minimax fit of 2^f on [-0.5, 0.5] under relative error (Remez exchange; the fit is reproduced
+// by block_sparse_long_causal_b200/exp2_fit.py); max relative error 7.5e-5, far below the bf16
+// rounding of P (2^-9). 2^n is applied by adding n to the exponent field: because
+// (0x4B400000 << 23) wraps to 0 in 32 bits, the shifted bits of x + 1.5*2^23 are exactly n << 23.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  const uint64_t xc = f2_make(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f2_make(12582912.f, 12582912.f);
+  const uint64_t t = fadd2(xc, magic);
+  const uint64_t f = fsub2(xc, fsub2(t, magic));
+  uint64_t q = ffma2(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
+  q = ffma2(q, f, f2_make(kExp2C1, kExp2C1));
+  q = ffma2(q, f, f2_make(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  return f2_make(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
 __device__ __forceinline__ void dev_flag(int32_t* dev_status, int bits) {
   if (dev_status) atomicOr(dev_status, bits);
 }

@@ -80,5 +80,6 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st);
 cudaError_t launch_search(const SearchParams& p, cudaStream_t st);
 cudaError_t launch_validate(const ValidateParams& p, cudaStream_t st);
 cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st);
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, long long n, cudaStream_t st);
 
 }  // namespace fp

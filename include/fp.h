@@ -126,6 +126,12 @@ FP_API fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k
 FP_API fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices,
                             int32_t* dev_status, void* stream);
 
+/* Self-test of the attention softmax's two exp2 paths (a repository test hook; the pages have no
+ * counterpart): for i < n, y_poly[i] = the FMA-pipe polynomial 2^x[i] (degree-3 minimax on the
+ * fractional part, inputs below -126 clamped) and y_mufu[i] = the hardware ex2.approx 2^x[i].
+ * x, y_poly, y_mufu: device float32 [n]. */
+FP_API fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream);
+
 /* Message for the last non-OK status returned on this thread (never NULL). */
 FP_API const char* fp_last_error(void);
 

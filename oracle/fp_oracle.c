@@ -85,11 +85,13 @@ int64_t orc_index_elems(const int32_t* cu, int S, int B, int Hq) {
 /* ---------------------------------------------------------------- pool ----------------------- */
 /* x: bf16 bits [T, H, d]; out: [NB, H, d] block means. Returns 0. */
 int orc_pool(const uint16_t* x, const int32_t* cu, int S, int H, int d, int B, double* out) {
-    int64_t gb = 0;
+    int64_t gb0 = 0;
     for (int s = 0; s < S; ++s) {
         int64_t start = cu[s], L = cu[s + 1] - cu[s];
         int64_t nb = blocks_of(L, B);
-        for (int64_t b = 0; b < nb; ++b, ++gb) {
+#pragma omp parallel for schedule(static)
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t gb = gb0 + b;
             int64_t t0 = start + b * B;
             int64_t t1 = start + ((b + 1) * B < L ? (b + 1) * B : L); /* partial last block */
             double n = (double)(t1 - t0);
@@ -101,6 +103,7 @@ int orc_pool(const uint16_t* x, const int32_t* cu, int S, int H, int d, int B, d
                 }
             }
         }
+        gb0 += nb;
     }
     return 0;
 }

@@ -91,3 +91,28 @@ def test_llama3_8b_L32768(tau):
     x = synth.make_inputs(w)
     rows = sample_rows(x["cu_seqlens"], w.hq, 192, seed=1)
     _check_case(x, w.hq, w.hkv, w.block, tau, rows=rows)
+
+
+def test_exp2_polynomial_error_bound():
+    """The FMA-pipe exp2 (degree-3 minimax, relative error 7.5e-5 by construction) against exact
+    2^x in fp64 and against the hardware ex2.approx, over the softmax's input range."""
+    import torch
+    import block_sparse_long_causal_b200 as fp
+    x = np.concatenate([np.linspace(-126.0, 8.0, 2_000_001), np.arange(-126, 9), np.arange(-126, 9) + 0.5,
+                        [0.0, -0.0, 1e-8, -1e-8]]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yp, ym = torch.empty_like(xd), torch.empty_like(xd)
+    fp.selftest_exp2(xd, yp, ym)
+    torch.cuda.synchronize()
+    exact = np.exp2(x.astype(np.float64))
+    rel_poly = np.abs(yp.cpu().numpy().astype(np.float64) / exact - 1.0)
+    rel_mufu = np.abs(ym.cpu().numpy().astype(np.float64) / exact - 1.0)
+    assert rel_poly.max() <= 1e-4, rel_poly.max()
+    assert rel_mufu.max() <= 1e-5, rel_mufu.max()
+    # below the clamp the polynomial returns 2^-126 times its value at the clamp, never garbage
+    xs = torch.tensor([-200.0, -1e30, float("-inf")], device="cuda")
+    yp2, ym2 = torch.empty_like(xs), torch.empty_like(xs)
+    fp.selftest_exp2(xs, yp2, ym2)
+    torch.cuda.synchronize()
+    v = yp2.cpu().numpy()
+    assert (v >= 0).all() and (v <= 2.0 ** -125).all()
