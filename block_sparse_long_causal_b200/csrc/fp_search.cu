@@ -89,52 +89,61 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
 // ---------------------------------------------------------------------------------- search ----
 // CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows (q-head, block) that
 // all share the pooled keys of kv-head g (GQA). Row r: head offset r % G, block offset r / G.
-// Warp w owns rows [8w, 8w+8); lane = key block j within a chunk of 32.
-// Pass 1: row max m_i and row min of s_ij over j <= i.
+// Scores are a register-tiled outer product over d: thread (rg, jg) owns rows 4rg..4rg+3 and key
+// blocks 4jg..4jg+3 of a 64-block chunk; pooled queries and keys sit transposed in shared memory
+// so every step of d is two 16-byte shared loads for 16 FMAs.
+// Pass 1: row max m_i and row min of s_ij over j <= i (scores stay in registers).
 // If min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
 // same decision the per-block test would take) and the row is written as 0..i directly.
-// Otherwise pass 2 recomputes the scores chunk by chunk and emits the kept blocks in order.
+// Otherwise pass 2 recomputes the chunk scores, stages them in shared memory, and one warp per row
+// emits the kept blocks in ascending order with ballot/popc compaction.
 constexpr int kSearchThreads = 256;
 constexpr int kSearchRows = 64;
-constexpr int kKChunk = 32;
-constexpr int kKStride = kHeadDim + 4;  // padded row (floats) -> conflict-free float4 reads
+constexpr int kKChunk = 64;
+constexpr int kTStride = kSearchRows + 4;  // transposed row stride (floats); 16-byte aligned
 
 struct SearchSmem {
-  float q[kSearchRows][kHeadDim];
-  float k[kKChunk][kKStride];
+  float qT[kHeadDim][kTStride];   // pooled queries, [d][row]
+  float kT[kHeadDim][kTStride];   // pooled keys of the current chunk, [d][j]
+  float sc[kSearchRows][kKChunk + 1];
   int cu[kMaxSeqs + 1], cb[kMaxSeqs + 1], ct[kMaxSeqs + 1];
   long long ib[kMaxSeqs + 1];
   int ok;
   int need_pass2;
 };
 
+// kT[d][jr] = kbar[gb0 + j0 + jr][g][d] (zero past jmax). Lane <-> key block so that the transposed
+// shared stores are conflict free; the loads are 16-byte pieces of L2-resident rows.
 __device__ __forceinline__ void load_k_chunk(SearchSmem& sm, const float* kp, int gb0, int g, int hkv, int j0,
                                              int jmax) {
-  // 32 rows x 128 floats = 1024 float4; 256 threads x 4
   for (int e = threadIdx.x; e < kKChunk * (kHeadDim / 4); e += kSearchThreads) {
-    const int jr = e / (kHeadDim / 4), c4 = e % (kHeadDim / 4);
+    const int jr = e % kKChunk, d4 = e / kKChunk;
     const int j = j0 + jr;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j <= jmax) v = reinterpret_cast<const float4*>(kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim)[c4];
-    *reinterpret_cast<float4*>(&sm.k[jr][c4 * 4]) = v;
+    if (j <= jmax) v = reinterpret_cast<const float4*>(kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim)[d4];
+    sm.kT[4 * d4 + 0][jr] = v.x;
+    sm.kT[4 * d4 + 1][jr] = v.y;
+    sm.kT[4 * d4 + 2][jr] = v.z;
+    sm.kT[4 * d4 + 3][jr] = v.w;
   }
 }
 
-// Dot products of the warp's 8 rows with key block (lane) of the current chunk.
-__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int row0, int lane, float (&acc)[8]) {
+// acc[a][b] = q_row(4rg+a) . k_block(4jg+b) over the full head dim.
+__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int rg, int jg, float (&acc)[4][4]) {
 #pragma unroll
-  for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < kHeadDim; c += 4) {
-    const float4 kv = *reinterpret_cast<const float4*>(&sm.k[lane][c]);
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const float4 qv = *reinterpret_cast<const float4*>(&sm.q[row0 + r][c]);
-      acc[r] = fmaf(qv.x, kv.x, acc[r]);
-      acc[r] = fmaf(qv.y, kv.y, acc[r]);
-      acc[r] = fmaf(qv.z, kv.z, acc[r]);
-      acc[r] = fmaf(qv.w, kv.w, acc[r]);
-    }
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 8
+  for (int d = 0; d < kHeadDim; ++d) {
+    const float4 qv = *reinterpret_cast<const float4*>(&sm.qT[d][4 * rg]);
+    const float4 kv = *reinterpret_cast<const float4*>(&sm.kT[d][4 * jg]);
+    const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float k4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(q4[a], k4[b], acc[a][b]);
   }
 }
 
@@ -151,6 +160,8 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
   }
   const int G = p.group, TI = p.rows_blocks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = warp * 2 + (lane >> 4);   // row group: rows 4rg..4rg+3
+  const int jg = lane & 15;                // key-block group: blocks 4jg..4jg+3 of a chunk
   const int NB = p.seq.total_blocks;
 
   const int num_tiles = sm.ct[S];
@@ -167,68 +178,87 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
 
     __syncthreads();  // previous tile done with shared memory
     for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
-      const int r = e / (kHeadDim / 4), c4 = e % (kHeadDim / 4);
+      const int r = e % kSearchRows, d4 = e / kSearchRows;
       const int i = i0 + r / G, h = g * G + r % G;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < TI * G && i <= i_last)
-        v = reinterpret_cast<const float4*>(p.q_pool + ((long long)(gb0 + i) * p.hq + h) * kHeadDim)[c4];
-      *reinterpret_cast<float4*>(&sm.q[r][c4 * 4]) = v;
+        v = reinterpret_cast<const float4*>(p.q_pool + ((long long)(gb0 + i) * p.hq + h) * kHeadDim)[d4];
+      sm.qT[4 * d4 + 0][r] = v.x;
+      sm.qT[4 * d4 + 1][r] = v.y;
+      sm.qT[4 * d4 + 2][r] = v.z;
+      sm.qT[4 * d4 + 3][r] = v.w;
     }
     if (threadIdx.x == 0) sm.need_pass2 = 0;
 
-    const int row0 = warp * 8;
-    int row_i[8], row_h[8];
+    // this thread's 4 rows (for the register tile) ...
+    int ti[4];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int rr = row0 + r;
-      row_i[r] = (rr < TI * G) ? i0 + rr / G : -1;
-      if (row_i[r] > i_last) row_i[r] = -1;
-      row_h[r] = g * G + rr % G;
+    for (int a = 0; a < 4; ++a) {
+      const int r = 4 * rg + a;
+      ti[a] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
     }
-    const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
-                              max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
-
-    float mx[8], mn[8];
+    const int t_imax = max(max(ti[0], ti[1]), max(ti[2], ti[3]));
+    float mx[4], mn[4];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) { mx[r] = -INFINITY; mn[r] = INFINITY; }
+    for (int a = 0; a < 4; ++a) { mx[a] = -INFINITY; mn[a] = INFINITY; }
 
     if (!p.keep_all) {
-      // ---- pass 1: row max / min of the pooled scores (kept in registers, never stored)
+      // ---- pass 1: row max / min of the pooled scores
       for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
         __syncthreads();
         load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
         __syncthreads();
-        if (j0 > warp_imax) continue;
-        float acc[8];
-        chunk_scores(sm, row0, lane, acc);
-        const int j = j0 + lane;
+        if (j0 > t_imax) continue;
+        float acc[4][4];
+        chunk_scores(sm, rg, jg, acc);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (j <= row_i[r]) {
-            const float sc = acc[r] * p.inv_sqrt_d;
-            mx[r] = fmaxf(mx[r], sc);
-            mn[r] = fminf(mn[r], sc);
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            if (j0 + 4 * jg + b <= ti[a]) {
+              const float sc = acc[a][b] * p.inv_sqrt_d;
+              mx[a] = fmaxf(mx[a], sc);
+              mn[a] = fminf(mn[a], sc);
+            }
           }
+      }
+      // reduce over the 16 threads (jg) sharing these rows
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          mx[a] = fmaxf(mx[a], __shfl_xor_sync(0xffffffffu, mx[a], o));
+          mn[a] = fminf(mn[a], __shfl_xor_sync(0xffffffffu, mn[a], o));
         }
       }
+      // publish per-row (max, min) for the emitting warps
+      __syncthreads();
+      if (jg == 0) {
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
-          mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
+        for (int a = 0; a < 4; ++a) {
+          sm.sc[4 * rg + a][0] = mx[a];
+          sm.sc[4 * rg + a][1] = mn[a];
         }
       }
     }
+    __syncthreads();
 
-    // rows whose every causal block passes are written as 0..i without recomputation
+    // ... and the emission rows: warp w emits rows 8w..8w+7
+    int row_i[8], row_h[8];
+    float rmx[8];
     bool all_keep[8];
     bool warp_needs = false;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      all_keep[r] = p.keep_all || (mn[r] - mx[r] >= p.log_tau);
+      const int rr = warp * 8 + r;
+      row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
+      row_h[r] = g * G + rr % G;
+      rmx[r] = p.keep_all ? 0.f : sm.sc[rr][0];
+      all_keep[r] = p.keep_all || (sm.sc[rr][1] - rmx[r] >= p.log_tau);
       if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
     }
+    const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
+                              max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
     if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
 
 #pragma unroll
@@ -255,18 +285,28 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
       __syncthreads();
       load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
       __syncthreads();
+      if (j0 <= t_imax) {
+        float acc[4][4];
+        chunk_scores(sm, rg, jg, acc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) sm.sc[4 * rg + a][4 * jg + b] = acc[a][b] * p.inv_sqrt_d;
+      }
+      __syncthreads();
       if (!warp_needs || j0 > warp_imax) continue;
-      float acc[8];
-      chunk_scores(sm, row0, lane, acc);
-      const int j = j0 + lane;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (row_i[r] < 0 || all_keep[r] || j0 > row_i[r]) continue;
-        const float sc = acc[r] * p.inv_sqrt_d;
-        const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || sc - mx[r] >= p.log_tau);
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
-        cnt[r] += __popc(bal);
+#pragma unroll
+        for (int h2 = 0; h2 < kKChunk; h2 += 32) {
+          const int j = j0 + h2 + lane;
+          const float sc = sm.sc[warp * 8 + r][h2 + lane];
+          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || sc - rmx[r] >= p.log_tau);
+          const unsigned bal = __ballot_sync(0xffffffffu, keep);
+          if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
+          cnt[r] += __popc(bal);
+        }
       }
     }
     if (lane == 0) {
