@@ -89,14 +89,15 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
 // ---------------------------------------------------------------------------------- search ----
 // CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows (q-head, block) that
 // all share the pooled keys of kv-head g (GQA). Row r: head offset r % G, block offset r / G.
-// Scores are a register-tiled outer product over d: thread (rg, jg) owns rows 4rg..4rg+3 and key
-// blocks 4jg..4jg+3 of a 64-block chunk; pooled queries and keys sit transposed in shared memory
-// so every step of d is two 16-byte shared loads for 16 FMAs.
+// Warp w owns rows 8w..8w+7 and lane l owns key blocks j0+2l, j0+2l+1 of a 64-block chunk; the
+// scores are a register-tiled outer product over d with pooled queries and keys transposed in
+// shared memory: per step of d, two broadcast 16-byte loads (8 rows, same for the whole warp) and
+// one 8-byte load per lane feed 16 FMAs, so the loop is bound by the FMA pipe, not shared memory.
 // Pass 1: row max m_i and row min of s_ij over j <= i (scores stay in registers).
 // If min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
 // same decision the per-block test would take) and the row is written as 0..i directly.
-// Otherwise pass 2 recomputes the chunk scores, stages them in shared memory, and one warp per row
-// emits the kept blocks in ascending order with ballot/popc compaction.
+// Otherwise pass 2 recomputes the scores and emits kept blocks in ascending order with two ballots
+// per row and chunk (even and odd key blocks) and popc prefix counts.
 constexpr int kSearchThreads = 256;
 constexpr int kSearchRows = 64;
 constexpr int kKChunk = 64;
@@ -105,7 +106,6 @@ constexpr int kTStride = kSearchRows + 4;  // transposed row stride (floats); 16
 struct SearchSmem {
   float qT[kHeadDim][kTStride];   // pooled queries, [d][row]
   float kT[kHeadDim][kTStride];   // pooled keys of the current chunk, [d][j]
-  float sc[kSearchRows][kKChunk + 1];
   int cu[kMaxSeqs + 1], cb[kMaxSeqs + 1], ct[kMaxSeqs + 1];
   long long ib[kMaxSeqs + 1];
   int ok;
@@ -128,22 +128,21 @@ __device__ __forceinline__ void load_k_chunk(SearchSmem& sm, const float* kp, in
   }
 }
 
-// acc[a][b] = q_row(4rg+a) . k_block(4jg+b) over the full head dim.
-__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int rg, int jg, float (&acc)[4][4]) {
+// acc[r][e] = q_row(8w+r) . k_block(2*lane+e) over the full head dim.
+__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int warp, int lane, float (&acc)[8][2]) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
 #pragma unroll 8
   for (int d = 0; d < kHeadDim; ++d) {
-    const float4 qv = *reinterpret_cast<const float4*>(&sm.qT[d][4 * rg]);
-    const float4 kv = *reinterpret_cast<const float4*>(&sm.kT[d][4 * jg]);
-    const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
-    const float k4[4] = {kv.x, kv.y, kv.z, kv.w};
+    const float4 qa = *reinterpret_cast<const float4*>(&sm.qT[d][8 * warp]);
+    const float4 qb = *reinterpret_cast<const float4*>(&sm.qT[d][8 * warp + 4]);
+    const float2 kv = *reinterpret_cast<const float2*>(&sm.kT[d][2 * lane]);
+    const float q8[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(q4[a], k4[b], acc[a][b]);
+    for (int r = 0; r < 8; ++r) {
+      acc[r][0] = fmaf(q8[r], kv.x, acc[r][0]);
+      acc[r][1] = fmaf(q8[r], kv.y, acc[r][1]);
+    }
   }
 }
 
@@ -160,9 +159,8 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
   }
   const int G = p.group, TI = p.rows_blocks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rg = warp * 2 + (lane >> 4);   // row group: rows 4rg..4rg+3
-  const int jg = lane & 15;                // key-block group: blocks 4jg..4jg+3 of a chunk
   const int NB = p.seq.total_blocks;
+  const unsigned lt_mask = (1u << lane) - 1u;
 
   const int num_tiles = sm.ct[S];
   for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -190,17 +188,18 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
     }
     if (threadIdx.x == 0) sm.need_pass2 = 0;
 
-    // this thread's 4 rows (for the register tile) ...
-    int ti[4];
+    int row_i[8], row_h[8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = 4 * rg + a;
-      ti[a] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+    for (int r = 0; r < 8; ++r) {
+      const int rr = warp * 8 + r;
+      row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
+      row_h[r] = g * G + rr % G;
     }
-    const int t_imax = max(max(ti[0], ti[1]), max(ti[2], ti[3]));
-    float mx[4], mn[4];
+    const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
+                              max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
+    float mx[8], mn[8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) { mx[a] = -INFINITY; mn[a] = INFINITY; }
+    for (int r = 0; r < 8; ++r) { mx[r] = -INFINITY; mn[r] = INFINITY; }
 
     if (!p.keep_all) {
       // ---- pass 1: row max / min of the pooled scores
@@ -208,59 +207,39 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
         __syncthreads();
         load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
         __syncthreads();
-        if (j0 > t_imax) continue;
-        float acc[4][4];
-        chunk_scores(sm, rg, jg, acc);
+        if (j0 > warp_imax) continue;
+        float acc[8][2];
+        chunk_scores(sm, warp, lane, acc);
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int r = 0; r < 8; ++r)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            if (j0 + 4 * jg + b <= ti[a]) {
-              const float sc = acc[a][b] * p.inv_sqrt_d;
-              mx[a] = fmaxf(mx[a], sc);
-              mn[a] = fminf(mn[a], sc);
+          for (int e = 0; e < 2; ++e) {
+            if (j0 + 2 * lane + e <= row_i[r]) {
+              const float sc = acc[r][e] * p.inv_sqrt_d;
+              mx[r] = fmaxf(mx[r], sc);
+              mn[r] = fminf(mn[r], sc);
             }
           }
       }
-      // reduce over the 16 threads (jg) sharing these rows
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
+      for (int r = 0; r < 8; ++r) {
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {
-          mx[a] = fmaxf(mx[a], __shfl_xor_sync(0xffffffffu, mx[a], o));
-          mn[a] = fminf(mn[a], __shfl_xor_sync(0xffffffffu, mn[a], o));
-        }
-      }
-      // publish per-row (max, min) for the emitting warps
-      __syncthreads();
-      if (jg == 0) {
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          sm.sc[4 * rg + a][0] = mx[a];
-          sm.sc[4 * rg + a][1] = mn[a];
+        for (int o = 16; o > 0; o >>= 1) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
+          mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
         }
       }
     }
-    __syncthreads();
 
-    // ... and the emission rows: warp w emits rows 8w..8w+7
-    int row_i[8], row_h[8];
-    float rmx[8];
+    // rows whose every causal block passes are written as 0..i without recomputation
     bool all_keep[8];
     bool warp_needs = false;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int rr = warp * 8 + r;
-      row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
-      row_h[r] = g * G + rr % G;
-      rmx[r] = p.keep_all ? 0.f : sm.sc[rr][0];
-      all_keep[r] = p.keep_all || (sm.sc[rr][1] - rmx[r] >= p.log_tau);
+      all_keep[r] = p.keep_all || (mn[r] - mx[r] >= p.log_tau);
       if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
     }
-    const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
-                              max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
     if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
-
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       if (row_i[r] < 0 || !all_keep[r]) continue;
@@ -280,33 +259,29 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
       cnt[r] = 0;
       base[r] = (row_i[r] >= 0) ? list_row(sm.cb, sm.ib, s, row_h[r], row_i[r]) : 0;
     }
-    const unsigned lt_mask = (1u << lane) - 1u;
     for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
       __syncthreads();
       load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
       __syncthreads();
-      if (j0 <= t_imax) {
-        float acc[4][4];
-        chunk_scores(sm, rg, jg, acc);
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) sm.sc[4 * rg + a][4 * jg + b] = acc[a][b] * p.inv_sqrt_d;
-      }
-      __syncthreads();
       if (!warp_needs || j0 > warp_imax) continue;
+      float acc[8][2];
+      chunk_scores(sm, warp, lane, acc);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (row_i[r] < 0 || all_keep[r] || j0 > row_i[r]) continue;
+        bool keep[2];
 #pragma unroll
-        for (int h2 = 0; h2 < kKChunk; h2 += 32) {
-          const int j = j0 + h2 + lane;
-          const float sc = sm.sc[warp * 8 + r][h2 + lane];
-          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || sc - rmx[r] >= p.log_tau);
-          const unsigned bal = __ballot_sync(0xffffffffu, keep);
-          if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
-          cnt[r] += __popc(bal);
+        for (int e = 0; e < 2; ++e) {
+          const int j = j0 + 2 * lane + e;
+          keep[e] = j <= row_i[r] && (j == 0 || j == row_i[r] || acc[r][e] * p.inv_sqrt_d - mx[r] >= p.log_tau);
         }
+        const unsigned b0 = __ballot_sync(0xffffffffu, keep[0]);
+        const unsigned b1 = __ballot_sync(0xffffffffu, keep[1]);
+        // ascending order j0 + 2l + e: entries before (l, e) are both of lanes < l, plus (l, 0) for e = 1
+        const int before = cnt[r] + __popc(b0 & lt_mask) + __popc(b1 & lt_mask);
+        if (keep[0]) p.indices[base[r] + before] = j0 + 2 * lane;
+        if (keep[1]) p.indices[base[r] + before + (keep[0] ? 1 : 0)] = j0 + 2 * lane + 1;
+        cnt[r] += __popc(b0) + __popc(b1);
       }
     }
     if (lane == 0) {
