@@ -95,14 +95,13 @@ fp_status cuda_status(cudaError_t e, const char* what) {
   return fail(FP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Limit of every bounded wait inside the attention kernel: 2 s, or FP_WAIT_LIMIT_MS (read at each
+// call, so a test can make the waits run out on purpose).
 uint64_t wait_limit_ns() {
-  static uint64_t v = [] {
-    const char* s = getenv("FP_WAIT_LIMIT_MS");
-    double ms = s ? atof(s) : 2000.0;
-    if (!(ms > 0.0)) ms = 2000.0;
-    return (uint64_t)(ms * 1e6);
-  }();
-  return v;
+  const char* s = getenv("FP_WAIT_LIMIT_MS");
+  double ms = s ? atof(s) : 2000.0;
+  if (!(ms > 0.0)) ms = 2000.0;
+  return (uint64_t)(ms * 1e6) > 0 ? (uint64_t)(ms * 1e6) : 1;
 }
 
 fp_status attn_common(const fp_problem* p, const void* q, const void* k, const void* v, const int32_t* counts,
@@ -140,6 +139,10 @@ fp_status attn_common(const fp_problem* p, const void* q, const void* k, const v
   a.lse = lse;
   a.dev_status = dev_status;
   a.wait_limit_ns = wait_limit_ns();
+  // test hook (bounded-wait failure path): FP_TEST_UNSIGNALLED_WAIT=1 makes the softmax warps wait
+  // on a barrier that nothing arrives on; the wait runs out, FP_DEV_TIMEOUT is set, the CTA unwinds
+  const char* tw = getenv("FP_TEST_UNSIGNALLED_WAIT");
+  a.test_unsignalled_wait = (tw && tw[0] == '1') ? 1 : 0;
   const int grid = (int)(tiles_ub < sm_count() ? tiles_ub : sm_count());
   return cuda_status(fp::launch_attn(a, grid, static_cast<cudaStream_t>(stream)), "attention launch");
 }

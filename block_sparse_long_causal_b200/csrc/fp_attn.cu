@@ -30,6 +30,8 @@ namespace fp {
 
 constexpr int kThreads = 192;
 constexpr unsigned kFull = 0xffffffffu;
+// Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
 // exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU: 3 of 8
 constexpr unsigned kPolyPairs = 0xA4u;
 constexpr uint32_t kTmemCols = 512;
@@ -48,8 +50,8 @@ struct Cfg {
   static constexpr uint32_t kOffV = kOffK + kStagesK * kKVBytes;
   static constexpr uint32_t kOffBar = kOffV + kStagesV * kKVBytes;
   // barriers: q_full, q_empty, k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2],
-  // o_done, o_final, drain
-  static constexpr int kNumBars = 2 + 2 * kStagesK + 2 * kStagesV + 4 + 3;
+  // o_done, o_final, drain, never (the test hook's barrier that nothing arrives on)
+  static constexpr int kNumBars = 2 + 2 * kStagesK + 2 * kStagesV + 4 + 4;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag, ok
   static constexpr uint32_t kOffTab = (kOffMisc + 16 + 15) & ~15u;
   static constexpr uint32_t kTabBytes = 3 * 4 * (kMaxSeqs + 1) + 8 * (kMaxSeqs + 1) + 16;
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t b_s_full0 = bar0 + 16 + 8 * (2 * C::kStagesK + 2 * C::kStagesV);
   const uint32_t b_p_full0 = b_s_full0 + 16;
   const uint32_t b_o_done = b_p_full0 + 16, b_o_final = b_o_done + 8, b_drain = b_o_final + 8;
+  const uint32_t b_never = b_drain + 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_ok = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -189,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     mbar_init(b_o_done, 1);
     mbar_init(b_o_final, 1);
     mbar_init(b_drain, 1);
+    mbar_init(b_never, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -214,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // =========================================================== TMA producer
     if (lane == 0) {
       uint32_t kit = 0, vit = 0;  // loads issued into the K / V rings
-      int tc = 0;
+      int tc = 0, tc_issued = 0;  // tiles started / Q loads issued
+      bool qissued = false;
       bool fail = false;
       for (int k = 0;; ++k, ++tc) {
         const int t = tile_of(k);
@@ -225,6 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         mbar_arrive_expect_tx(b_q_full, C::kQBytes);
         tma_load_2d(sQ, &p.tm_q, b_q_full, tl.h * kHeadDim, tl.row0);
         tma_load_2d(sQ + C::kSlabQ, &p.tm_q, b_q_full, tl.h * kHeadDim + 64, tl.row0);
+        ++tc_issued;
+        qissued = true;
         KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
         int j, mask, pending_v = -1;
         while (true) {
@@ -257,15 +264,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       if (fail) {
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
-        // let issued copies land before the CTA can exit
+        // let issued copies land before the CTA can exit (own, generous limit: copies always land)
         for (int i = 0; i < C::kStagesK; ++i) {
           const uint32_t n = kit > (uint32_t)i ? (kit - 1 - i) / C::kStagesK : 0;
-          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), n & 1, p.wait_limit_ns);
+          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), n & 1, kDrainLimitNs);
         }
         for (int i = 0; i < C::kStagesV; ++i) {
           const uint32_t n = vit > (uint32_t)i ? (vit - 1 - i) / C::kStagesV : 0;
-          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), n & 1, p.wait_limit_ns);
+          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), n & 1, kDrainLimitNs);
         }
+        if (qissued) mbar_wait(b_q_full, (uint32_t)(tc_issued - 1) & 1, kDrainLimitNs);
       }
     }
     __syncwarp();
@@ -335,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
       }
-      // all issued MMAs complete before TMEM is released
+      // all issued MMAs complete before TMEM is released (own, generous limit: MMAs always finish)
       mma_commit(b_drain);
-      mbar_wait(b_drain, 0, p.wait_limit_ns);
+      mbar_wait(b_drain, 0, kDrainLimitNs);
     }
     __syncwarp();
   } else {
@@ -350,6 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     int fc = 0;  // tiles with a non-empty kv list (phases of o_final)
     bool fail = false;
     bool bad_list = false;
+    if (p.test_unsignalled_wait && num_tiles > 0)
+      fail = __any_sync(kFull, !mbar_wait(b_never, 0, p.wait_limit_ns));
     for (int k = 0;; ++k) {
       const int t = tile_of(k);
       if (t >= num_tiles || fail) break;

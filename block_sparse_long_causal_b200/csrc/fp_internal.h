@@ -70,6 +70,7 @@ struct __align__(64) AttnParams {
   float* lse;                 // [Hq, T] or null
   int32_t* dev_status;
   uint64_t wait_limit_ns;
+  int32_t test_unsignalled_wait;  // test hook: softmax warps first wait on a barrier nothing signals
 };
 
 constexpr int kMaxSeqs = FP_MAX_SEQS;

@@ -89,64 +89,79 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
 // ---------------------------------------------------------------------------------- search ----
 // CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows (q-head, block) that
 // all share the pooled keys of kv-head g (GQA). Row r: head offset r % G, block offset r / G.
-// Warp w owns rows 8w..8w+7 and lane l owns key blocks j0+2l, j0+2l+1 of a 64-block chunk; the
-// scores are a register-tiled outer product over d with pooled queries and keys transposed in
-// shared memory: per step of d, two broadcast 16-byte loads (8 rows, same for the whole warp) and
-// one 8-byte load per lane feed 16 FMAs, so the loop is bound by the FMA pipe, not shared memory.
+// Pooled keys stream through shared memory in chunks of 64 blocks, double buffered with cp.async
+// (16-byte global->shared copies in flight while the previous chunk is scored). Warp w scores key
+// blocks 8w..8w+7 of a chunk (broadcast shared reads) against rows 2l, 2l+1 of lane l (pooled
+// queries transposed in shared memory): per 4 steps of d, 8 broadcast and 4 lane-private loads
+// feed 64 FMAs, so the loop is bound by the FMA pipe.
 // Pass 1: row max m_i and row min of s_ij over j <= i (scores stay in registers).
 // If min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
 // same decision the per-block test would take) and the row is written as 0..i directly.
-// Otherwise pass 2 recomputes the scores and emits kept blocks in ascending order with two ballots
-// per row and chunk (even and odd key blocks) and popc prefix counts.
+// Otherwise pass 2 recomputes the scores, stages them in shared memory, and one warp per 8 rows
+// emits the kept blocks in ascending order with ballot/popc compaction.
 constexpr int kSearchThreads = 256;
+constexpr int kSearchWarps = kSearchThreads / 32;
 constexpr int kSearchRows = 64;
-constexpr int kKChunk = 64;
-constexpr int kTStride = kSearchRows + 4;  // transposed row stride (floats); 16-byte aligned
+constexpr int kKChunk = 64;                  // key blocks per chunk (8 per warp)
+constexpr int kQTStride = kSearchRows + 4;   // transposed pooled-query row stride (floats)
+constexpr int kKStride = kHeadDim + 4;       // pooled-key row stride (floats), 16-byte aligned
 
 struct SearchSmem {
-  float qT[kHeadDim][kTStride];   // pooled queries, [d][row]
-  float kT[kHeadDim][kTStride];   // pooled keys of the current chunk, [d][j]
+  float k[2][kKChunk][kKStride];             // pooled keys, natural layout, two buffers
+  float qT[kHeadDim][kQTStride];             // pooled queries, [d][row]
+  float red[2][kSearchWarps][kSearchRows];   // per-warp row max / min
+  float sc[kSearchRows][kKChunk + 1];        // chunk scores for the emission pass
   int cu[kMaxSeqs + 1], cb[kMaxSeqs + 1], ct[kMaxSeqs + 1];
   long long ib[kMaxSeqs + 1];
   int ok;
   int need_pass2;
 };
 
-// kT[d][jr] = kbar[gb0 + j0 + jr][g][d] (zero past jmax). Lane <-> key block so that the transposed
-// shared stores are conflict free; the loads are 16-byte pieces of L2-resident rows.
-__device__ __forceinline__ void load_k_chunk(SearchSmem& sm, const float* kp, int gb0, int g, int hkv, int j0,
-                                             int jmax) {
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = smem_u32(dst);
+  const int n = valid ? 16 : 0;  // 0 source bytes -> 16 zero bytes
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all_but_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Issue the copies of chunk [j0, j0+64) of kv-head g's pooled keys into buffer `buf` (zero past jmax).
+__device__ __forceinline__ void issue_k_chunk(SearchSmem& sm, int buf, const float* kp, int gb0, int g, int hkv,
+                                              int j0, int jmax) {
   for (int e = threadIdx.x; e < kKChunk * (kHeadDim / 4); e += kSearchThreads) {
-    const int jr = e % kKChunk, d4 = e / kKChunk;
-    const int j = j0 + jr;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j <= jmax) v = reinterpret_cast<const float4*>(kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim)[d4];
-    sm.kT[4 * d4 + 0][jr] = v.x;
-    sm.kT[4 * d4 + 1][jr] = v.y;
-    sm.kT[4 * d4 + 2][jr] = v.z;
-    sm.kT[4 * d4 + 3][jr] = v.w;
+    const int jr = e / (kHeadDim / 4), c4 = e % (kHeadDim / 4);
+    const int j = min(j0 + jr, jmax);
+    cp_async16(&sm.k[buf][jr][4 * c4], kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim + 4 * c4, j0 + jr <= jmax);
   }
+  cp_async_commit();
 }
 
-// acc[r][e] = q_row(8w+r) . k_block(2*lane+e) over the full head dim.
-__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int warp, int lane, float (&acc)[8][2]) {
+// acc[e][b] = q_row(2*lane+e) . k_block(8*warp+b) over the full head dim.
+__device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int buf, int warp, int lane, float (&acc)[2][8]) {
 #pragma unroll
-  for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
-#pragma unroll 8
-  for (int d = 0; d < kHeadDim; ++d) {
-    const float4 qa = *reinterpret_cast<const float4*>(&sm.qT[d][8 * warp]);
-    const float4 qb = *reinterpret_cast<const float4*>(&sm.qT[d][8 * warp + 4]);
-    const float2 kv = *reinterpret_cast<const float2*>(&sm.kT[d][2 * lane]);
-    const float q8[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+  for (int e = 0; e < 2; ++e)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      acc[r][0] = fmaf(q8[r], kv.x, acc[r][0]);
-      acc[r][1] = fmaf(q8[r], kv.y, acc[r][1]);
+    for (int b = 0; b < 8; ++b) acc[e][b] = 0.f;
+#pragma unroll 2
+  for (int d = 0; d < kHeadDim; d += 4) {
+    float4 kv[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) kv[b] = *reinterpret_cast<const float4*>(&sm.k[buf][8 * warp + b][d]);
+#pragma unroll
+    for (int dd = 0; dd < 4; ++dd) {
+      const float2 q2 = *reinterpret_cast<const float2*>(&sm.qT[d + dd][2 * lane]);
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const float kk = dd == 0 ? kv[b].x : dd == 1 ? kv[b].y : dd == 2 ? kv[b].z : kv[b].w;
+        acc[0][b] = fmaf(q2.x, kk, acc[0][b]);
+        acc[1][b] = fmaf(q2.y, kk, acc[1][b]);
+      }
     }
   }
 }
 
-__global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchParams p) {
+__global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchParams p) {
   extern __shared__ __align__(16) unsigned char search_smem_raw[];
   SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
   if (!build_seq_tables(p.seq, sm.cu, sm.cb, sm.ct, sm.ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
@@ -173,8 +188,10 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
     const int i0 = it * TI;
     const int i_last = min(i0 + TI, nb) - 1;
     const int gb0 = sm.cb[s];
+    const int nchunks = i_last / kKChunk + 1;
 
     __syncthreads();  // previous tile done with shared memory
+    if (!p.keep_all) issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, 0, i_last);
     for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
       const int r = e % kSearchRows, d4 = e / kSearchRows;
       const int i = i0 + r / G, h = g * G + r % G;
@@ -188,57 +205,72 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
     }
     if (threadIdx.x == 0) sm.need_pass2 = 0;
 
+    // scoring rows of this lane
+    int li[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      li[e] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+    }
+    float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
+
+    if (!p.keep_all) {
+      // ---- pass 1: row max / min of the pooled scores
+      for (int c = 0; c < nchunks; ++c) {
+        const int j0 = c * kKChunk;
+        if (c + 1 < nchunks) {
+          __syncthreads();  // buffer (c+1)&1 no longer read
+          issue_k_chunk(sm, (c + 1) & 1, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
+          cp_async_wait_all_but_one();
+        } else {
+          cp_async_wait_all();
+        }
+        __syncthreads();
+        float acc[2][8];
+        chunk_scores(sm, c & 1, warp, lane, acc);
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+          for (int b = 0; b < 8; ++b) {
+            if (j0 + 8 * warp + b <= li[e]) {
+              const float sc = acc[e][b] * p.inv_sqrt_d;
+              mx[e] = fmaxf(mx[e], sc);
+              mn[e] = fminf(mn[e], sc);
+            }
+          }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sm.red[0][warp][2 * lane + e] = mx[e];
+        sm.red[1][warp][2 * lane + e] = mn[e];
+      }
+    }
+    __syncthreads();
+
+    // emission rows: warp w emits rows 8w..8w+7
     int row_i[8], row_h[8];
+    float rmx[8];
+    bool all_keep[8];
+    bool warp_needs = false;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int rr = warp * 8 + r;
       row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
       row_h[r] = g * G + rr % G;
+      float a = -INFINITY, b = INFINITY;
+      if (!p.keep_all) {
+#pragma unroll
+        for (int w = 0; w < kSearchWarps; ++w) {
+          a = fmaxf(a, sm.red[0][w][rr]);
+          b = fminf(b, sm.red[1][w][rr]);
+        }
+      }
+      rmx[r] = a;
+      all_keep[r] = p.keep_all || (b - a >= p.log_tau);
+      if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
     }
     const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
                               max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
-    float mx[8], mn[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) { mx[r] = -INFINITY; mn[r] = INFINITY; }
-
-    if (!p.keep_all) {
-      // ---- pass 1: row max / min of the pooled scores
-      for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
-        __syncthreads();
-        load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
-        __syncthreads();
-        if (j0 > warp_imax) continue;
-        float acc[8][2];
-        chunk_scores(sm, warp, lane, acc);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            if (j0 + 2 * lane + e <= row_i[r]) {
-              const float sc = acc[r][e] * p.inv_sqrt_d;
-              mx[r] = fmaxf(mx[r], sc);
-              mn[r] = fminf(mn[r], sc);
-            }
-          }
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
-          mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
-        }
-      }
-    }
-
-    // rows whose every causal block passes are written as 0..i without recomputation
-    bool all_keep[8];
-    bool warp_needs = false;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      all_keep[r] = p.keep_all || (mn[r] - mx[r] >= p.log_tau);
-      if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
-    }
     if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -259,29 +291,32 @@ __global__ void __launch_bounds__(kSearchThreads) search_kernel(const SearchPara
       cnt[r] = 0;
       base[r] = (row_i[r] >= 0) ? list_row(sm.cb, sm.ib, s, row_h[r], row_i[r]) : 0;
     }
-    for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int j0 = c * kKChunk;
       __syncthreads();
-      load_k_chunk(sm, p.k_pool, gb0, g, p.hkv, j0, i_last);
+      issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, j0, i_last);
+      cp_async_wait_all();
+      __syncthreads();
+      float acc[2][8];
+      chunk_scores(sm, 0, warp, lane, acc);
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) sm.sc[2 * lane + e][8 * warp + b] = acc[e][b] * p.inv_sqrt_d;
       __syncthreads();
       if (!warp_needs || j0 > warp_imax) continue;
-      float acc[8][2];
-      chunk_scores(sm, warp, lane, acc);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (row_i[r] < 0 || all_keep[r] || j0 > row_i[r]) continue;
-        bool keep[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + 2 * lane + e;
-          keep[e] = j <= row_i[r] && (j == 0 || j == row_i[r] || acc[r][e] * p.inv_sqrt_d - mx[r] >= p.log_tau);
+        for (int h2 = 0; h2 < kKChunk; h2 += 32) {
+          const int j = j0 + h2 + lane;
+          const float sc = sm.sc[warp * 8 + r][h2 + lane];
+          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || sc - rmx[r] >= p.log_tau);
+          const unsigned bal = __ballot_sync(0xffffffffu, keep);
+          if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
+          cnt[r] += __popc(bal);
         }
-        const unsigned b0 = __ballot_sync(0xffffffffu, keep[0]);
-        const unsigned b1 = __ballot_sync(0xffffffffu, keep[1]);
-        // ascending order j0 + 2l + e: entries before (l, e) are both of lanes < l, plus (l, 0) for e = 1
-        const int before = cnt[r] + __popc(b0 & lt_mask) + __popc(b1 & lt_mask);
-        if (keep[0]) p.indices[base[r] + before] = j0 + 2 * lane;
-        if (keep[1]) p.indices[base[r] + before + (keep[0] ? 1 : 0)] = j0 + 2 * lane + 1;
-        cnt[r] += __popc(b0) + __popc(b1);
       }
     }
     if (lane == 0) {
@@ -303,7 +338,7 @@ cudaError_t launch_search(const SearchParams& p, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = p.num_tiles < sms * 4 ? p.num_tiles : sms * 4;
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   if (grid <= 0) return cudaSuccess;
   search_kernel<<<grid, kSearchThreads, smem, st>>>(p);
   return cudaGetLastError();
