@@ -69,19 +69,24 @@ struct Tile {
   int gb0;          // global id of block 0 of the sequence
 };
 
+// Tile order inside a sequence: kv-head outermost, then query tile descending (longest causal rows
+// first), then the G q-heads of that kv-head. The CTAs running at the same time then stream the
+// K/V blocks of one kv-head, which stay in L2 while the G q-heads and neighbouring query tiles
+// reuse them.
 __device__ __forceinline__ Tile decode_tile(int t, const int* s_cu, const int* s_cb, const int* s_ct, int S,
-                                            int hq, int block) {
+                                            int hq, int group) {
   Tile x;
   x.s = find_seq(s_ct, S, t);
   const int local = t - s_ct[x.s];
   const int ntile = (s_ct[x.s + 1] - s_ct[x.s]) / hq;
-  x.qt = ntile - 1 - local / hq;
-  x.h = local % hq;
+  const int per_g = ntile * group;
+  const int g = local / per_g, rem = local % per_g;
+  x.qt = ntile - 1 - rem / group;
+  x.h = g * group + rem % group;
   x.row0 = s_cu[x.s] + x.qt * kTileM;
   x.len = s_cu[x.s + 1] - s_cu[x.s];
   x.nb = s_cb[x.s + 1] - s_cb[x.s];
   x.gb0 = s_cb[x.s];
-  (void)block;
   return x;
 }
 
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       for (int k = 0;; ++k, ++tc) {
         const int t = tile_of(k);
         if (t >= num_tiles || fail) break;
-        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, BK);
+        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
         const int g = tl.h / p.group;
         if (!mbar_wait(b_q_empty, (tc & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
         mbar_arrive_expect_tx(b_q_full, C::kQBytes);
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       for (int k = 0;; ++k, ++tc) {
         const int t = tile_of(k);
         if (t >= num_tiles || fail) break;
-        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, BK);
+        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
         KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
         if (!mbar_wait(b_q_full, tc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
@@ -363,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     for (int k = 0;; ++k) {
       const int t = tile_of(k);
       if (t >= num_tiles || fail) break;
-      const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, BK);
+      const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
       KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
       const int qpos = tl.qt * kTileM + r;    // local query position of this row
       float m_run = -INFINITY, l_run = 0.f;
