@@ -2,56 +2,73 @@
 //
 // FlashPrefill, skill summary page, "Architecture Overview" ("Physical Index Jumping": attention
 // visits only the blocks named by the index lists) and the FlashPrefill V2 abstract (block-sparse
-// prefill operator with warp specialisation; a dense baseline built the same way). The online
-// softmax is the standard flash-attention recurrence.
+// prefill operator with PackGQA memory access, warp specialisation and pingpong pipelining; a dense
+// baseline built the same way). The online softmax is the standard flash-attention recurrence.
 //
-// Design (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: Q tile (128 rows x 128 d, bf16, 128B swizzle, two 64-column slabs),
-//               K and V tiles of B keys in rings of kStagesK / kStagesV slots; K/V coordinates
-//               come straight from the index lists ("physical index jumping").
-//   warp 1      tcgen05 issuer (one thread): S = Q K^T (M=128, N=B, K=16 steps) into TMEM, then
-//               O += P V with P read from TMEM (A operand) and V from shared memory (MN-major B).
-//               Owns the TMEM allocation (512 columns: S0 | S1 | O).
-//   warps 2-5   softmax: thread r owns query row r of the tile (its TMEM lane). Loads S from TMEM,
-//               applies the causal mask on diagonal tiles, keeps a running max in log2 units and
-//               only rescales O (in TMEM) when the max grows by more than 2^8 (the stale max is
-//               exact because numerator and denominator share it), writes P as bf16 into the S
-//               columns it came from, and finally normalises O and stores it (and the LSE).
-// S/P are double buffered so the QK^T of block n+1 overlaps the softmax of block n.
-// GQA: tiles are ordered (query tile descending, then q-head), so the G q-heads sharing a kv-head
-// run on neighbouring CTAs at the same time and their K/V tiles come from L2 after the first read.
-// Block size 64: a 128-row tile holds two query blocks; the kv iteration is the ascending union of
-// both lists, and a per-half bit masks rows of the block whose list lacks the current kv block.
-// Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, drains and returns.
+// Design (one persistent CTA per SM, 12 warps in three warpgroups):
+//   WG0  warp 0: TMA producer. Per work unit two Q tiles (128 rows x 128 d, bf16, 128B swizzle),
+//                then K and V tiles of B keys in rings of kStages slots; K/V coordinates come
+//                straight from the index lists ("physical index jumping").
+//        warp 1: allocates 512 TMEM columns (S0 | S1 | O0 | O1) and issues tcgen05.mma from one
+//                thread: S_k = Q_k K^T (M=128, N=B, K=16 steps, both operands K-major SW128 smem
+//                descriptors) and O_k += P_k V (P_k read from TMEM as the A operand, V an MN-major
+//                SW128 descriptor), in the pingpong order PV0(n-1) QK0(n) PV1(n-1) QK1(n).
+//        warps 2-3: idle (they only give their registers to the softmax warpgroups).
+//   WG1, WG2  softmax of slot 0 / slot 1: thread r owns query row r of its slot's tile (its TMEM
+//                lane): tcgen05.ld of S, causal mask on diagonal tiles, running max in log2 units,
+//                exp2 split between MUFU and an FMA-pipe polynomial, P packed to bf16 back into the
+//                S columns, lazy O rescale (only when the max grows by more than 2^8), final
+//                normalisation and the bf16 store of O and the LSE.
+// Registers: setmaxnreg moves WG0 down to 104 and WG1/WG2 up to 200 per thread
+// (128*104 + 256*200 = 384*168, the launch allocation of __launch_bounds__(384, 1)).
+//
+// A work unit pairs two Q tiles that read the same K/V stream, so each K/V tile is loaded once
+// into shared memory for both (GQA packing):
+//   G = Hq/Hkv even: q-heads (2p, 2p+1) of one kv-head, same query tile;
+//   G odd:           one q-head, query tiles (2m+1, 2m) (the last may run alone).
+// The kv iteration is the ascending union of the slots' lists (two per slot when B = 64, where a
+// 128-row tile holds two query blocks); a per-(slot, half) bit masks rows whose list lacks the
+// current block, so different lists stay exact.
+// Because QK_k(n) is issued after PV_k(n-1) and tcgen05.commit tracks all earlier MMAs, a slot
+// that sees S_k(n) may rescale O_k without waiting: PV_k(n-1) has already completed.
+// Units are ordered kv-head outermost, then by descending query tile, so concurrent CTAs stream
+// the K/V of one kv-head (L2 resident) and the longest causal rows start first.
+// Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, lets issued copies and MMAs
+// finish, frees TMEM and returns.
 #include "fp_internal.h"
 #include "fp_seq.cuh"
 
 namespace fp {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr unsigned kFull = 0xffffffffu;
-// Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
-constexpr uint64_t kDrainLimitNs = 1000000000ull;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kRegsCtl = 104;       // WG0 (producer, MMA, idle)
+constexpr int kRegsSoftmax = 200;  // WG1, WG2
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * 168,
+              "register split must equal the launch allocation");
 // exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU: 3 of 8
 constexpr unsigned kPolyPairs = 0xA4u;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0, kTmemO = 256;
+// Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+__device__ __forceinline__ uint32_t tmem_s(int k) { return 128u * k; }
+__device__ __forceinline__ uint32_t tmem_o(int k) { return 256u + 128u * k; }
 
 template <int BK>
 struct Cfg {
-  static constexpr int kStagesK = BK == 128 ? 3 : 4;
-  static constexpr int kStagesV = BK == 128 ? 2 : 4;
-  static constexpr uint32_t kQBytes = kTileM * kHeadDim * 2;        // 32 KB
+  static constexpr int kStages = BK == 128 ? 2 : 4;                // K ring and V ring slots
+  static constexpr uint32_t kQBytes = kTileM * kHeadDim * 2;        // 32 KB per slot
   static constexpr uint32_t kKVBytes = BK * kHeadDim * 2;           // one K or V tile
   static constexpr uint32_t kSlabQ = kTileM * 128;                  // 64 cols x 2 B x rows
   static constexpr uint32_t kSlabKV = BK * 128;
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kQBytes;
-  static constexpr uint32_t kOffV = kOffK + kStagesK * kKVBytes;
-  static constexpr uint32_t kOffBar = kOffV + kStagesV * kKVBytes;
+  static constexpr uint32_t kOffK = 2 * kQBytes;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
+  static constexpr uint32_t kOffBar = kOffV + kStages * kKVBytes;
   // barriers: q_full, q_empty, k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2],
-  // o_done, o_final, drain, never (the test hook's barrier that nothing arrives on)
-  static constexpr int kNumBars = 2 + 2 * kStagesK + 2 * kStagesV + 4 + 4;
+  // o_final[2], drain, never (the test hook's barrier that nothing arrives on)
+  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag, ok
   static constexpr uint32_t kOffTab = (kOffMisc + 16 + 15) & ~15u;
   static constexpr uint32_t kTabBytes = 3 * 4 * (kMaxSeqs + 1) + 8 * (kMaxSeqs + 1) + 16;
@@ -60,98 +77,122 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHeadDim, 0, 1);
 };
 
-// ------------------------------------------------------------------------ tile schedule --------
-struct Tile {
-  int s, qt, h;     // sequence, 128-row query tile (local), q-head
-  int row0;         // first token (global) of the tile
-  int len;          // sequence length
-  int nb;           // blocks of the sequence
-  int gb0;          // global id of block 0 of the sequence
+// ------------------------------------------------------------------------ work units ----------
+struct Unit {
+  int s, g;         // sequence, kv-head
+  int nslot;        // 1 or 2 active Q slots
+  int qt[2], h[2];  // per slot: 128-row query tile (local), q-head
+  int seq0;         // first token of the sequence
+  int len, nb, gb0; // sequence length, its blocks, global id of its block 0
 };
 
-// Tile order inside a sequence: kv-head outermost, then query tile descending (longest causal rows
-// first), then the G q-heads of that kv-head. The CTAs running at the same time then stream the
-// K/V blocks of one kv-head, which stay in L2 while the G q-heads and neighbouring query tiles
-// reuse them.
-__device__ __forceinline__ Tile decode_tile(int t, const int* s_cu, const int* s_cb, const int* s_ct, int S,
-                                            int hq, int group) {
-  Tile x;
-  x.s = find_seq(s_ct, S, t);
-  const int local = t - s_ct[x.s];
-  const int ntile = (s_ct[x.s + 1] - s_ct[x.s]) / hq;
-  const int per_g = ntile * group;
-  const int g = local / per_g, rem = local % per_g;
-  x.qt = ntile - 1 - rem / group;
-  x.h = g * group + rem % group;
-  x.row0 = s_cu[x.s] + x.qt * kTileM;
-  x.len = s_cu[x.s + 1] - s_cu[x.s];
-  x.nb = s_cb[x.s + 1] - s_cb[x.s];
-  x.gb0 = s_cb[x.s];
-  return x;
+// Unit order inside a sequence: kv-head outermost, then descending query tile, then the q-head
+// pairs (G even) or q-heads (G odd) of that kv-head.
+__device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s_cb, const int* s_ct, int S,
+                                            int group) {
+  Unit u;
+  u.s = find_seq(s_ct, S, t);
+  const int local = t - s_ct[u.s];
+  u.seq0 = s_cu[u.s];
+  u.len = s_cu[u.s + 1] - u.seq0;
+  u.nb = s_cb[u.s + 1] - s_cb[u.s];
+  u.gb0 = s_cb[u.s];
+  const int ntile = (u.len + kTileM - 1) / kTileM;
+  if ((group & 1) == 0) {
+    const int pairs = group / 2;
+    const int per_g = ntile * pairs;
+    u.g = local / per_g;
+    const int rem = local % per_g;
+    const int qt = ntile - 1 - rem / pairs;
+    const int pr = rem % pairs;
+    u.nslot = 2;
+    u.qt[0] = u.qt[1] = qt;
+    u.h[0] = u.g * group + 2 * pr;
+    u.h[1] = u.h[0] + 1;
+  } else {
+    const int np = (ntile + 1) / 2;
+    const int per_g = np * group;
+    u.g = local / per_g;
+    const int rem = local % per_g;
+    const int m = np - 1 - rem / group;
+    const int h = u.g * group + rem % group;
+    u.h[0] = u.h[1] = h;
+    if (2 * m + 1 < ntile) {
+      u.nslot = 2;
+      u.qt[0] = 2 * m + 1;
+      u.qt[1] = 2 * m;
+    } else {
+      u.nslot = 1;
+      u.qt[0] = u.qt[1] = 2 * m;
+    }
+  }
+  return u;
 }
 
-// k-th tile of this CTA in a boustrophedon order over the grid (balances the descending sizes).
-__device__ __forceinline__ int tile_of(int k) {
+// k-th unit of this CTA in a boustrophedon order over the grid (balances the descending sizes).
+__device__ __forceinline__ int unit_of(int k) {
   const int g = gridDim.x;
   return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
 // ---------------------------------------------------------------------- kv iteration -----------
-// Ascending union of up to two lists (A: query block a_blk, B: query block b_blk = a_blk + 1 when
-// B == 64). Entries outside [0, own block] are skipped (and reported by the softmax role).
+// Ascending union of up to four lists: list q = 2*slot + half (half = second query block of a
+// 128-row tile when B = 64). Entries outside [0, own block] are skipped (and reported).
 struct KvIter {
-  const int32_t* la;
-  const int32_t* lb;
-  int na, nbn, ia, ib, lima, limb;
+  const int32_t* l[4];
+  int n[4], i[4], lim[4];
   bool dense;
   bool bad;
 
-  __device__ __forceinline__ int peek(const int32_t* l, int n, int& i, int lim) {
-    while (i < n) {
-      const int x = dense ? i : __ldg(l + i);
-      if (x >= 0 && x <= lim) return x;
+  __device__ __forceinline__ int peek(int q) {
+    while (i[q] < n[q]) {
+      const int x = dense ? i[q] : __ldg(l[q] + i[q]);
+      if (x >= 0 && x <= lim[q]) return x;
       bad = true;
-      ++i;
+      ++i[q];
     }
     return 0x7fffffff;
   }
   __device__ __forceinline__ bool next(int& j, int& mask) {
-    const int ja = peek(la, na, ia, lima);
-    const int jb = peek(lb, nbn, ib, limb);
-    if (ja == 0x7fffffff && jb == 0x7fffffff) return false;
-    j = min(ja, jb);
-    mask = (ja == j ? 1 : 0) | (jb == j ? 2 : 0);
-    if (ja == j) ++ia;
-    if (jb == j) ++ib;
+    int v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = peek(q);
+    j = min(min(v[0], v[1]), min(v[2], v[3]));
+    if (j == 0x7fffffff) return false;
+    mask = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (v[q] == j) {
+        mask |= 1 << q;
+        ++i[q];
+      }
     return true;
   }
 };
 
 template <int BK>
-__device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Tile& t, const int* s_cb, const long long* s_ib) {
+__device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, const int* s_cb,
+                                            const long long* s_ib) {
   KvIter it;
-  it.ia = it.ib = 0;
   it.bad = false;
   it.dense = p.dense != 0;
   constexpr int per = kTileM / BK;  // query blocks per tile
-  const int a_blk = t.qt * per;
-  const int b_blk = (per == 2 && a_blk + 1 < t.nb) ? a_blk + 1 : -1;
-  it.lima = a_blk;
-  it.limb = b_blk;
-  if (it.dense) {
-    it.la = it.lb = nullptr;
-    it.na = a_blk + 1;
-    it.nbn = b_blk >= 0 ? b_blk + 1 : 0;
-  } else {
-    const int NB = p.seq.total_blocks;
-    it.la = p.indices + list_row(s_cb, s_ib, t.s, t.h, a_blk);
-    it.na = min(max(__ldg(p.counts + (long long)t.h * NB + t.gb0 + a_blk), 0), a_blk + 1);
-    if (b_blk >= 0) {
-      it.lb = p.indices + list_row(s_cb, s_ib, t.s, t.h, b_blk);
-      it.nbn = min(max(__ldg(p.counts + (long long)t.h * NB + t.gb0 + b_blk), 0), b_blk + 1);
+  const int NB = p.seq.total_blocks;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k = q >> 1, hf = q & 1;
+    const int blk = u.qt[k] * per + hf;
+    const bool exists = k < u.nslot && hf < per && blk < u.nb;
+    it.i[q] = 0;
+    it.lim[q] = blk;
+    it.l[q] = nullptr;
+    it.n[q] = 0;
+    if (!exists) continue;
+    if (it.dense) {
+      it.n[q] = blk + 1;
     } else {
-      it.lb = nullptr;
-      it.nbn = 0;
+      it.l[q] = p.indices + list_row(s_cb, s_ib, u.s, u.h[k], blk);
+      it.n[q] = min(max(__ldg(p.counts + (long long)u.h[k] * NB + u.gb0 + blk), 0), blk + 1);
     }
   }
   return it;
@@ -166,16 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
   const uint32_t bar0 = sbase + C::kOffBar;
-  // barrier addresses
   const uint32_t b_q_full = bar0, b_q_empty = bar0 + 8;
   auto b_k_full = [&](int i) { return bar0 + 16 + 8 * i; };
-  auto b_k_empty = [&](int i) { return bar0 + 16 + 8 * (C::kStagesK + i); };
-  auto b_v_full = [&](int i) { return bar0 + 16 + 8 * (2 * C::kStagesK + i); };
-  auto b_v_empty = [&](int i) { return bar0 + 16 + 8 * (2 * C::kStagesK + C::kStagesV + i); };
-  const uint32_t b_s_full0 = bar0 + 16 + 8 * (2 * C::kStagesK + 2 * C::kStagesV);
+  auto b_k_empty = [&](int i) { return bar0 + 16 + 8 * (C::kStages + i); };
+  auto b_v_full = [&](int i) { return bar0 + 16 + 8 * (2 * C::kStages + i); };
+  auto b_v_empty = [&](int i) { return bar0 + 16 + 8 * (3 * C::kStages + i); };
+  const uint32_t b_s_full0 = bar0 + 16 + 8 * (4 * C::kStages);
   const uint32_t b_p_full0 = b_s_full0 + 16;
-  const uint32_t b_o_done = b_p_full0 + 16, b_o_final = b_o_done + 8, b_drain = b_o_final + 8;
-  const uint32_t b_never = b_drain + 8;
+  const uint32_t b_o_final0 = b_p_full0 + 16;
+  const uint32_t b_drain = b_o_final0 + 16, b_never = b_drain + 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_ok = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -186,16 +226,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   s_ib = reinterpret_cast<long long*>(((uintptr_t)s_ib + 7) & ~(uintptr_t)7);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
   const int S = p.seq.num_seqs;
+  const bool even_g = (p.group & 1) == 0;
 
   if (threadIdx.x == 0) {
     mbar_init(b_q_full, 1);
     mbar_init(b_q_empty, 1);
-    for (int i = 0; i < C::kStagesK; ++i) { mbar_init(b_k_full(i), 1); mbar_init(b_k_empty(i), 1); }
-    for (int i = 0; i < C::kStagesV; ++i) { mbar_init(b_v_full(i), 1); mbar_init(b_v_empty(i), 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(b_s_full0 + 8 * i, 1); mbar_init(b_p_full0 + 8 * i, 128); }
-    mbar_init(b_o_done, 1);
-    mbar_init(b_o_final, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(b_k_full(i), 1);
+      mbar_init(b_k_empty(i), 1);
+      mbar_init(b_v_full(i), 1);
+      mbar_init(b_v_empty(i), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(b_s_full0 + 8 * k, 1);
+      mbar_init(b_p_full0 + 8 * k, 128);
+      mbar_init(b_o_final0 + 8 * k, 1);
+    }
     mbar_init(b_drain, 1);
     mbar_init(b_never, 1);
     *s_abort = 0;
@@ -210,59 +258,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
   }
-  const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, kTileM, p.hq, s_ok, p.dev_status) &&
+  // unit table: G even -> Hq/2 units per 128 query rows; G odd -> Hq units per 256 query rows
+  const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, even_g ? kTileM : 2 * kTileM,
+                                   even_g ? p.hq / 2 : p.hq, s_ok, p.dev_status) &&
                   (p.dense || s_ib[S] == p.index_elems);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   if (!ok && threadIdx.x == 0 && !p.dense) dev_flag(p.dev_status, kDevBadProblem);
-  const int num_tiles = ok ? s_ct[S] : 0;
+  const int num_units = ok ? s_ct[S] : 0;
 
+  if (wg == 0) {
+    // register budget of the producer / MMA / idle warpgroup (all four warps execute it)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+  }
   if (warp == 0) {
     // =========================================================== TMA producer
     if (lane == 0) {
       uint32_t kit = 0, vit = 0;  // loads issued into the K / V rings
-      int tc = 0, tc_issued = 0;  // tiles started / Q loads issued
-      bool qissued = false;
+      int uc = 0, q_issued = 0;   // units started / Q loads issued
       bool fail = false;
-      for (int k = 0;; ++k, ++tc) {
-        const int t = tile_of(k);
-        if (t >= num_tiles || fail) break;
-        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
-        const int g = tl.h / p.group;
-        if (!mbar_wait(b_q_empty, (tc & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-        mbar_arrive_expect_tx(b_q_full, C::kQBytes);
-        tma_load_2d(sQ, &p.tm_q, b_q_full, tl.h * kHeadDim, tl.row0);
-        tma_load_2d(sQ + C::kSlabQ, &p.tm_q, b_q_full, tl.h * kHeadDim + 64, tl.row0);
-        ++tc_issued;
-        qissued = true;
-        KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
-        int j, mask, pending_v = -1;
-        while (true) {
-          const bool more = itr.next(j, mask);
-          if (more) {  // K of this block
-            const int st = kit % C::kStagesK;
-            if (!mbar_wait(b_k_empty(st), ((kit / C::kStagesK) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-            mbar_arrive_expect_tx(b_k_full(st), C::kKVBytes);
-            const uint32_t dst = sK + st * C::kKVBytes;
-            const int y = tl.row0 - tl.qt * kTileM + j * BK;
-            tma_load_2d(dst, &p.tm_k, b_k_full(st), g * kHeadDim, y);
-            tma_load_2d(dst + C::kSlabKV, &p.tm_k, b_k_full(st), g * kHeadDim + 64, y);
-            ++kit;
-          }
-          if (pending_v >= 0) {  // V of the previous block (consumed after the next QK^T)
-            const int st = vit % C::kStagesV;
-            if (!mbar_wait(b_v_empty(st), ((vit / C::kStagesV) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-            mbar_arrive_expect_tx(b_v_full(st), C::kKVBytes);
-            const uint32_t dst = sV + st * C::kKVBytes;
-            const int y = tl.row0 - tl.qt * kTileM + pending_v * BK;
-            tma_load_2d(dst, &p.tm_v, b_v_full(st), g * kHeadDim, y);
-            tma_load_2d(dst + C::kSlabKV, &p.tm_v, b_v_full(st), g * kHeadDim + 64, y);
-            ++vit;
-          }
-          if (!more) break;
-          pending_v = j;
+      for (int k = 0;; ++k, ++uc) {
+        const int t = unit_of(k);
+        if (t >= num_units || fail) break;
+        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+        if (!mbar_wait(b_q_empty, (uc & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+        mbar_arrive_expect_tx(b_q_full, C::kQBytes * u.nslot);
+        for (int sl = 0; sl < u.nslot; ++sl) {
+          const int y = u.seq0 + u.qt[sl] * kTileM;
+          tma_load_2d(sQ + sl * C::kQBytes, &p.tm_q, b_q_full, u.h[sl] * kHeadDim, y);
+          tma_load_2d(sQ + sl * C::kQBytes + C::kSlabQ, &p.tm_q, b_q_full, u.h[sl] * kHeadDim + 64, y);
+        }
+        ++q_issued;
+        KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
+        int j, mask;
+        while (itr.next(j, mask)) {
+          const int y = u.seq0 + j * BK;
+          const int ks = kit % C::kStages;
+          if (!mbar_wait(b_k_empty(ks), ((kit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+          mbar_arrive_expect_tx(b_k_full(ks), C::kKVBytes);
+          tma_load_2d(sK + ks * C::kKVBytes, &p.tm_k, b_k_full(ks), u.g * kHeadDim, y);
+          tma_load_2d(sK + ks * C::kKVBytes + C::kSlabKV, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, y);
+          ++kit;
+          const int vs = vit % C::kStages;
+          if (!mbar_wait(b_v_empty(vs), ((vit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+          mbar_arrive_expect_tx(b_v_full(vs), C::kKVBytes);
+          tma_load_2d(sV + vs * C::kKVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, y);
+          tma_load_2d(sV + vs * C::kKVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, y);
+          ++vit;
           if (*s_abort) { fail = true; break; }
         }
       }
@@ -270,78 +314,89 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
         // let issued copies land before the CTA can exit (own, generous limit: copies always land)
-        for (int i = 0; i < C::kStagesK; ++i) {
-          const uint32_t n = kit > (uint32_t)i ? (kit - 1 - i) / C::kStagesK : 0;
-          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), n & 1, kDrainLimitNs);
+        for (int i = 0; i < C::kStages; ++i) {
+          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), ((kit - 1 - i) / C::kStages) & 1, kDrainLimitNs);
+          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), ((vit - 1 - i) / C::kStages) & 1, kDrainLimitNs);
         }
-        for (int i = 0; i < C::kStagesV; ++i) {
-          const uint32_t n = vit > (uint32_t)i ? (vit - 1 - i) / C::kStagesV : 0;
-          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), n & 1, kDrainLimitNs);
-        }
-        if (qissued) mbar_wait(b_q_full, (uint32_t)(tc_issued - 1) & 1, kDrainLimitNs);
+        if (q_issued > 0) mbar_wait(b_q_full, (uint32_t)(q_issued - 1) & 1, kDrainLimitNs);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // =========================================================== tcgen05 issuer
     if (lane == 0) {
-      uint32_t it = 0, vit = 0;
-      int tc = 0;
+      uint32_t kit = 0, vit = 0;  // K / V tiles consumed
+      uint32_t cnt[2] = {0, 0};   // items processed per slot (S/P barrier phases)
+      int uc = 0;
       bool fail = false;
-      auto pv = [&](uint32_t m, bool first) -> bool {
-        const uint32_t b = m & 1;
-        if (!mbar_wait(b_p_full0 + 8 * b, (m >> 1) & 1, p.wait_limit_ns)) return false;
-        const int st = vit % C::kStagesV;
-        if (!mbar_wait(b_v_full(st), (vit / C::kStagesV) & 1, p.wait_limit_ns)) return false;
+      // O_k += P_k V for the slot's previous item (V tile vit % kStages)
+      auto pv = [&](int k, bool first) -> bool {
+        if (!mbar_wait(b_p_full0 + 8 * k, (cnt[k] - 1) & 1, p.wait_limit_ns)) return false;
+        const int vs = vit % C::kStages;
+        if (!mbar_wait(b_v_full(vs), (vit / C::kStages) & 1, p.wait_limit_ns)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + st * C::kKVBytes;
+        const uint32_t vbase = sV + vs * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSlabKV, 1024);
-          mma_ts(tmem + kTmemO, tmem + kTmemS + 128 * b + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + tmem_o(k), tmem + tmem_s(k) + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(b_v_empty(st));
-        mma_commit(b_o_done);
-        ++vit;
         return true;
       };
-      for (int k = 0;; ++k, ++tc) {
-        const int t = tile_of(k);
-        if (t >= num_tiles || fail) break;
-        const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
-        KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
-        if (!mbar_wait(b_q_full, tc & 1, p.wait_limit_ns)) { fail = true; break; }
+      // S_k = Q_k K^T for the current item (K tile at kbase)
+      auto qk = [&](int k, uint32_t kbase) {
+        const uint32_t qbase = sQ + k * C::kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
+          const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * C::kSlabQ + koff, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * C::kSlabKV + koff, 16, 1024);
+          mma_ss(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_s_full0 + 8 * k);
+        ++cnt[k];
+      };
+      for (int k = 0;; ++k, ++uc) {
+        const int t = unit_of(k);
+        if (t >= num_units || fail) break;
+        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+        KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
+        if (!mbar_wait(b_q_full, uc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
         int j, mask, n = 0;
         bool more = itr.next(j, mask);
         while (more) {
-          const int st = it % C::kStagesK;
-          if (!mbar_wait(b_k_full(st), (it / C::kStagesK) & 1, p.wait_limit_ns)) { fail = true; break; }
+          const int ks = kit % C::kStages;
+          if (!mbar_wait(b_k_full(ks), (kit / C::kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
-          const uint32_t b = it & 1;
-          const uint32_t kbase = sK + st * C::kKVBytes;
-#pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
-            const uint64_t adesc = sdesc_sw128(sQ + (kk >> 2) * C::kSlabQ + koff, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * C::kSlabKV + koff, 16, 1024);
-            mma_ss(tmem + kTmemS + 128 * b, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t kbase = sK + ks * C::kKVBytes;
+          if (n > 0 && !pv(0, n == 1)) { fail = true; break; }
+          qk(0, kbase);
+          if (u.nslot == 2) {
+            if (n > 0 && !pv(1, n == 1)) { fail = true; break; }
+            qk(1, kbase);
           }
-          mma_commit(b_s_full0 + 8 * b);
-          mma_commit(b_k_empty(st));
+          if (n > 0) {  // both PVs of the previous item are issued: release its V tile
+            mma_commit(b_v_empty(vit % C::kStages));
+            ++vit;
+          }
+          mma_commit(b_k_empty(ks));
+          ++kit;
           more = itr.next(j, mask);
           if (!more) mma_commit(b_q_empty);
-          if (n > 0 && !pv(it - 1, n == 1)) { fail = true; break; }
-          ++it;
           ++n;
           if (*s_abort) { fail = true; break; }
         }
         if (fail) break;
         if (n > 0) {
-          if (!pv(it - 1, n == 1)) { fail = true; break; }
-          mma_commit(b_o_final);
+          if (!pv(0, n == 1)) { fail = true; break; }
+          if (u.nslot == 2 && !pv(1, n == 1)) { fail = true; break; }
+          mma_commit(b_v_empty(vit % C::kStages));
+          ++vit;
+          mma_commit(b_o_final0);
+          if (u.nslot == 2) mma_commit(b_o_final0 + 8);
         } else {
-          mma_commit(b_q_empty);  // empty list: release Q without touching O
+          mma_commit(b_q_empty);  // empty kv list: release Q without touching O
         }
       }
       if (fail) {
@@ -353,61 +408,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_wait(b_drain, 0, kDrainLimitNs);
     }
     __syncwarp();
-  } else {
+  } else if (wg >= 1) {
     // =========================================================== softmax / correction / epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int slot = wg - 1;
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
-    const int r = q4 * 32 + lane;             // row of the tile owned by this thread
+    const int r = q4 * 32 + lane;             // row of the slot's tile owned by this thread
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const int half = r / BK;                  // query block (within the tile) of this row
-    uint32_t it = 0;
-    int fc = 0;  // tiles with a non-empty kv list (phases of o_final)
+    const int half = (BK == 64) ? (r >> 6) : 0;
+    const int mbit = 2 * slot + half;         // this row's bit in the iteration mask
+    const uint32_t s_col = tmem + lane_off + tmem_s(slot), o_col = tmem + lane_off + tmem_o(slot);
+    const uint32_t b_s_full = b_s_full0 + 8 * slot, b_p_full = b_p_full0 + 8 * slot;
+    const uint32_t b_o_final = b_o_final0 + 8 * slot;
+    uint32_t cnt = 0;  // items processed by this slot (S/P barrier phases)
+    int fc = 0;        // units of this slot with a non-empty list (o_final phases)
     bool fail = false;
     bool bad_list = false;
-    if (p.test_unsignalled_wait && num_tiles > 0)
+    if (p.test_unsignalled_wait && num_units > 0)
       fail = __any_sync(kFull, !mbar_wait(b_never, 0, p.wait_limit_ns));
     for (int k = 0;; ++k) {
-      const int t = tile_of(k);
-      if (t >= num_tiles || fail) break;
-      const Tile tl = decode_tile(t, s_cu, s_cb, s_ct, S, p.hq, p.group);
-      KvIter itr = make_iter<BK>(p, tl, s_cb, s_ib);
-      const int qpos = tl.qt * kTileM + r;    // local query position of this row
+      const int t = unit_of(k);
+      if (t >= num_units || fail) break;
+      const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+      if (slot >= u.nslot) continue;          // this slot idles for the unit (same for the CTA)
+      KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
+      const int qpos = u.qt[slot] * kTileM + r;  // local query position of this row
       float m_run = -INFINITY, l_run = 0.f;
       int j, mask, n = 0;
       while (itr.next(j, mask)) {
-        const uint32_t b = it & 1;
-        // tcgen05.ld/st are warp-collective: every branch around them is made warp-uniform
-        if (__any_sync(kFull, !mbar_wait(b_s_full0 + 8 * b, (it >> 1) & 1, p.wait_limit_ns))) { fail = true; break; }
+        // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
+        if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
         uint32_t sr[BK];
 #pragma unroll
         for (int c = 0; c < BK; c += 32)
-          tmem_ld32(tmem + lane_off + kTmemS + 128 * b + c, *reinterpret_cast<uint32_t(*)[32]>(&sr[c]));
+          tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sr[c]));
         tmem_wait_ld();
-        // causal mask (diagonal tiles) and the per-half list mask (B = 64)
-        const int valid = ((mask >> (kTileM / BK == 2 ? half : 0)) & 1) ? (qpos - j * BK) : -1;
-        const bool masked = valid < BK - 1;   // this row needs element masking on this tile
+        // causal mask (diagonal tiles) and the list mask of this row's query block
+        const int valid = ((mask >> mbit) & 1) ? (qpos - j * BK) : -1;
+        const bool masked = valid < BK - 1;
         float mx;
-        if (masked) {
+        {
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (masked) {
 #pragma unroll
-          for (int c = 0; c < BK; ++c) {
-            const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
-            sr[c] = __float_as_uint(v);
-            m4[c & 3] = fmaxf(m4[c & 3], v);
-          }
-          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-        } else {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            for (int c = 0; c < BK; ++c) {
+              const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
+              sr[c] = __float_as_uint(v);
+              m4[c & 3] = fmaxf(m4[c & 3], v);
+            }
+          } else {
 #pragma unroll
-          for (int c = 0; c < BK; c += 8) {
+            for (int c = 0; c < BK; c += 8) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-              m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
+              for (int a = 0; a < 4; ++a)
+                m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
+            }
           }
           mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         }
-        const float m_tile = mx * p.scale_log2;
-        const float m_new = fmaxf(m_run, m_tile);
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
         // grow the reference max only when it rises by more than 2^8 (lazy rescale); the stale
         // max is exact because the numerator and the denominator share it
         const bool grow = m_new > m_run + 8.0f;
@@ -418,14 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         l_run *= alpha;
         if (n > 0 && __any_sync(kFull, grow)) {
-          // O must hold PV_{n-1} before it is rescaled (lanes that did not grow scale by 1)
-          if (__any_sync(kFull, !mbar_wait(b_o_done, (it - 1) & 1, p.wait_limit_ns))) { fail = true; break; }
-          tc_fence_after();
+          // S_k(n) was committed after PV_k(n-1): O_k is complete; lanes that did not grow scale by 1
           const uint64_t a2 = f2_make(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < kHeadDim; c += 32) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_off + kTmemO + c, o);
+            tmem_ld32(o_col + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
@@ -434,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
               o[e] = __float_as_uint(lo);
               o[e + 1] = __float_as_uint(hi);
             }
-            tmem_st32(tmem + lane_off + kTmemO + c, o);
+            tmem_st32(o_col + c, o);
           }
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
@@ -453,8 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             pk[c / 2] = pack_bf16x2(p0, p1);
           }
         } else {
-          // split exp2 between MUFU and the FMA-pipe polynomial (pairs whose index has a bit in
-          // kPolyPairs use the polynomial) so that neither unit alone bounds the softmax
+          // split exp2 between MUFU and the FMA-pipe polynomial so neither unit alone bounds it
 #pragma unroll
           for (int c = 0; c < BK; c += 2) {
             const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
@@ -480,21 +537,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
 #pragma unroll
         for (int c = 0; c < BK / 2; c += 32)
-          tmem_st32(tmem + lane_off + kTmemS + 128 * b + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
+          tmem_st32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(b_p_full0 + 8 * b);
-        ++it;
+        mbar_arrive(b_p_full);
+        ++cnt;
         ++n;
       }
       bad_list |= itr.bad;
       if (__any_sync(kFull, fail || *s_abort)) { fail = true; break; }
-      const bool row_ok = qpos < tl.len;
+      const bool row_ok = qpos < u.len;
+      const long long row = (long long)u.seq0 + qpos;
       if (n == 0) {  // empty kv list (malformed input): zero output, LSE -inf
         if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + ((long long)(tl.row0 + r) * p.hq + tl.h) * kHeadDim);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (row * p.hq + u.h[slot]) * kHeadDim);
           for (int c = 0; c < kHeadDim / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-          if (p.lse) p.lse[(long long)tl.h * p.seq.total_tokens + tl.row0 + r] = -INFINITY;
+          if (p.lse) p.lse[(long long)u.h[slot] * p.seq.total_tokens + row] = -INFINITY;
         }
         continue;
       }
@@ -503,11 +561,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       ++fc;
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      uint16_t* orow = p.out + ((long long)(tl.row0 + r) * p.hq + tl.h) * kHeadDim;
+      uint16_t* orow = p.out + (row * p.hq + u.h[slot]) * kHeadDim;
 #pragma unroll 1
       for (int c = 0; c < kHeadDim; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + kTmemO + c, o);
+        tmem_ld32(o_col + c, o);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
@@ -523,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       if (row_ok && p.lse) {
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        p.lse[(long long)tl.h * p.seq.total_tokens + tl.row0 + r] =
+        p.lse[(long long)u.h[slot] * p.seq.total_tokens + row] =
             l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
       }
       tc_fence_before();
@@ -545,7 +603,8 @@ template <int BK>
 static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BK>::kSmem);
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BK>::kSmem);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
