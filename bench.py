@@ -47,6 +47,23 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu record, if it was taken on these exact sources."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for rel in rec["sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        if rec["kernel"] != kernel or rec["workload"] != workload or h.hexdigest() != rec["sources_sha256"]:
+            return None
+        return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    except Exception:
+        return None
+
+
 def kept_flops(counts: np.ndarray, cu: np.ndarray, B: int, d: int) -> tuple[float, float]:
     """(effective FLOPs over kept blocks, dense-equivalent causal FLOPs).
 
@@ -309,7 +326,8 @@ def run_ours(args):
         "speedup_vs_own_dense": round(dense_ms / ms_step, 4) if dense_ms else None,
         "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": round(attn_tflops, 2),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tflops / peak_tf, 4),
-                     "peak_source": f"{pk['source']} bf16 sustained", "traffic": None},
+                     "peak_source": f"{pk['source']} bf16 sustained",
+                     "traffic": measured_traffic(f"attn_kernel<{w.block}>", w.name)},
         "search_roofline": None,
         "gpu_launches": 3 * args.steps,
         "dev_status": status,

@@ -52,6 +52,9 @@ SMALL = [
     ((513,), 4, 4, 64, 0.5, 3.0),
     ((64, 65, 127, 191), 4, 1, 64, 0.8, 3.0),
     ((2048,), 8, 1, 128, 0.0, 1.0),
+    ((900, 385), 6, 2, 128, 0.6, 3.0),      # G = 3: units pair query tiles of one head
+    ((1000, 129), 3, 1, 64, 0.7, 3.0),      # G = 3 with B = 64 (four lists per unit)
+    ((513,), 2, 2, 128, 0.3, 3.0),          # G = 1, odd tile count (last unit runs one slot)
 ]
 
 
