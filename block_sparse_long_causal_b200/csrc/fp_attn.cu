@@ -51,6 +51,14 @@ static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * 168,
 constexpr unsigned kPolyPairs = 0xA4u;
 // Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
+// Item ring: the producer merges the index lists once and publishes each kv item as
+// (block << 4 | row-mask bits) in a shared ring, one mbarrier per entry; -1 ends a unit. The
+// producer can never lead the slowest reader by more than 2 * (kStages + 3) entries (a K load waits for
+// the QK of item n - kStages, which needs both slots' P of the item before), so the ring keeps a
+// parity wait from ever seeing a phase two ahead (32 leaves room for one-item units, which add an
+// end marker per item).
+constexpr int kRing = 32;
+constexpr int kItemEnd = -1;
 
 __device__ __forceinline__ uint32_t tmem_s(int k) { return 128u * k; }
 __device__ __forceinline__ uint32_t tmem_o(int k) { return 256u + 128u * k; }
@@ -67,10 +75,11 @@ struct Cfg {
   static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
   static constexpr uint32_t kOffBar = kOffV + kStages * kKVBytes;
   // barriers: q_full, q_empty, k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2],
-  // o_final[2], drain, never (the test hook's barrier that nothing arrives on)
-  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2;
+  // o_final[2], drain, never (the test hook's barrier that nothing arrives on), item[kRing]
+  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2 + kRing;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag, ok
-  static constexpr uint32_t kOffTab = (kOffMisc + 16 + 15) & ~15u;
+  static constexpr uint32_t kOffRing = kOffMisc + 16;               // kRing int32 item entries
+  static constexpr uint32_t kOffTab = (kOffRing + 4 * kRing + 15) & ~15u;
   static constexpr uint32_t kTabBytes = 3 * 4 * (kMaxSeqs + 1) + 8 * (kMaxSeqs + 1) + 16;
   static constexpr uint32_t kSmem = kOffTab + kTabBytes + 1024;     // + alignment slack
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BK, 0, 0);
@@ -216,6 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t b_p_full0 = b_s_full0 + 16;
   const uint32_t b_o_final0 = b_p_full0 + 16;
   const uint32_t b_drain = b_o_final0 + 16, b_never = b_drain + 8;
+  auto b_item = [&](uint32_t x) { return b_never + 8 + 8 * (x % kRing); };
+  volatile int* s_item = reinterpret_cast<volatile int*>(smem + C::kOffRing);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_ok = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -246,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     mbar_init(b_drain, 1);
     mbar_init(b_never, 1);
+    for (int i = 0; i < kRing; ++i) mbar_init(b_item(i), 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -277,8 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // =========================================================== TMA producer
     if (lane == 0) {
       uint32_t kit = 0, vit = 0;  // loads issued into the K / V rings
+      uint32_t xit = 0;           // item-ring entries published
       int uc = 0, q_issued = 0;   // units started / Q loads issued
       bool fail = false;
+      bool bad_list = false;
       for (int k = 0;; ++k, ++uc) {
         const int t = unit_of(k);
         if (t >= num_units || fail) break;
@@ -293,7 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         ++q_issued;
         KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
         int j, mask;
-        while (itr.next(j, mask)) {
+        while (true) {
+          const bool more = itr.next(j, mask);
+          s_item[xit % kRing] = more ? (j << 4) | mask : kItemEnd;  // publish the item (or the unit's end)
+          mbar_arrive(b_item(xit));
+          ++xit;
+          if (!more) break;
           const int y = u.seq0 + j * BK;
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_empty(ks), ((kit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
@@ -309,7 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           ++vit;
           if (*s_abort) { fail = true; break; }
         }
+        bad_list |= itr.bad;
       }
+      if (bad_list) dev_flag(p.dev_status, kDevBadList);
       if (fail) {
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
@@ -356,15 +377,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         mma_commit(b_s_full0 + 8 * k);
         ++cnt[k];
       };
+      uint32_t xit = 0;  // item-ring entries read
+      auto read_item = [&](int& e) -> bool {
+        if (!mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns)) return false;
+        e = s_item[xit % kRing];
+        ++xit;
+        return true;
+      };
       for (int k = 0;; ++k, ++uc) {
         const int t = unit_of(k);
         if (t >= num_units || fail) break;
         const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
-        KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
         if (!mbar_wait(b_q_full, uc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
-        int j, mask, n = 0;
-        bool more = itr.next(j, mask);
+        int e, n = 0;
+        if (!read_item(e)) { fail = true; break; }
+        bool more = e != kItemEnd;
         while (more) {
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_full(ks), (kit / C::kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
@@ -382,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
           mma_commit(b_k_empty(ks));
           ++kit;
-          more = itr.next(j, mask);
+          if (!read_item(e)) { fail = true; break; }
+          more = e != kItemEnd;
           if (!more) mma_commit(b_q_empty);
           ++n;
           if (*s_abort) { fail = true; break; }
@@ -421,21 +450,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const uint32_t b_s_full = b_s_full0 + 8 * slot, b_p_full = b_p_full0 + 8 * slot;
     const uint32_t b_o_final = b_o_final0 + 8 * slot;
     uint32_t cnt = 0;  // items processed by this slot (S/P barrier phases)
+    uint32_t xit = 0;  // item-ring entries read
     int fc = 0;        // units of this slot with a non-empty list (o_final phases)
     bool fail = false;
-    bool bad_list = false;
     if (p.test_unsignalled_wait && num_units > 0)
       fail = __any_sync(kFull, !mbar_wait(b_never, 0, p.wait_limit_ns));
     for (int k = 0;; ++k) {
       const int t = unit_of(k);
       if (t >= num_units || fail) break;
       const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
-      if (slot >= u.nslot) continue;          // this slot idles for the unit (same for the CTA)
-      KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
+      const bool active = slot < u.nslot;     // an idle slot only consumes the unit's ring entries
       const int qpos = u.qt[slot] * kTileM + r;  // local query position of this row
       float m_run = -INFINITY, l_run = 0.f;
-      int j, mask, n = 0;
-      while (itr.next(j, mask)) {
+      int n = 0;
+      while (true) {
+        if (__any_sync(kFull, !mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns))) { fail = true; break; }
+        const int e = s_item[xit % kRing];
+        ++xit;
+        if (e == kItemEnd) break;
+        if (!active) continue;
+        const int j = e >> 4, mask = e & 15;
         // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
         if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
@@ -544,8 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         ++cnt;
         ++n;
       }
-      bad_list |= itr.bad;
       if (__any_sync(kFull, fail || *s_abort)) { fail = true; break; }
+      if (!active) continue;
       const bool row_ok = qpos < u.len;
       const long long row = (long long)u.seq0 + qpos;
       if (n == 0) {  // empty kv list (malformed input): zero output, LSE -inf
@@ -590,7 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       *s_abort = 1;
       dev_flag(p.dev_status, kDevTimeout);
     }
-    if (bad_list && r == 0) dev_flag(p.dev_status, kDevBadList);
   }
 
   tc_fence_before();
