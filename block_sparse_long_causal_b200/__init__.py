@@ -8,6 +8,7 @@ Entry points mirror the C ABI in include/fp.h:
     problem(...)            -> Problem (fp_problem_init)
     block_pool(...)         -> fp_block_pool
     block_search(...)       -> fp_block_search
+    block_pool_search(...)  -> fp_block_pool_search (steps 1 + 2 fused)
     block_sparse_attn(...)  -> fp_block_sparse_attn
     dense_attn(...)         -> fp_dense_attn
     validate_lists(...)     -> fp_validate_lists
@@ -27,7 +28,8 @@ LIB_PATH = os.path.join(_HERE, "libfp.so")
 FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 1, 2, 3, 4
 FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
 FP_MAX_SEQS = 1024
-EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_sparse_attn", "fp_dense_attn",
+EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_pool_search", "fp_block_sparse_attn",
+            "fp_dense_attn",
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version")
 
 
@@ -54,6 +56,7 @@ def _load():
         "fp_problem_init": [P, vp, i32, vp, i32, i32, i32, i32],
         "fp_block_pool": [P, vp, vp, vp, vp, vp],
         "fp_block_search": [P, vp, vp, f32, vp, vp, vp, vp],
+        "fp_block_pool_search": [P, vp, vp, f32, vp, vp, vp, vp, vp, vp],
         "fp_block_sparse_attn": [P, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_dense_attn": [P, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_validate_lists": [P, vp, vp, vp, vp],
@@ -138,6 +141,11 @@ def block_search(p: Problem, q_pool, k_pool, tau: float, counts, indices, dev_st
                                 _ptr(dev_status), _stream(stream)))
 
 
+def block_pool_search(p: Problem, q, k, tau: float, q_pool, k_pool, counts, indices, dev_status=None, stream=None):
+    _check(_lib.fp_block_pool_search(p.ref, _ptr(q), _ptr(k), float(tau), _ptr(q_pool), _ptr(k_pool), _ptr(counts),
+                                     _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
 def block_sparse_attn(p: Problem, q, k, v, counts, indices, softmax_scale: float, out, lse=None, dev_status=None,
                       stream=None):
     _check(_lib.fp_block_sparse_attn(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(counts), _ptr(indices),
@@ -175,9 +183,13 @@ class SparsePrefill:
         self.lse = torch.empty((hq, max(p.total_tokens, 1)), dtype=torch.float32, device=device) if with_lse else None
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=device)
 
-    def search(self, q, k, tau: float, stream=None):
-        block_pool(self.p, q, k, self.q_pool, self.k_pool, stream)
-        block_search(self.p, self.q_pool, self.k_pool, tau, self.counts, self.indices, self.dev_status, stream)
+    def search(self, q, k, tau: float, stream=None, fused: bool = True):
+        if fused:
+            block_pool_search(self.p, q, k, tau, self.q_pool, self.k_pool, self.counts, self.indices,
+                              self.dev_status, stream)
+        else:
+            block_pool(self.p, q, k, self.q_pool, self.k_pool, stream)
+            block_search(self.p, self.q_pool, self.k_pool, tau, self.counts, self.indices, self.dev_status, stream)
 
     def attend(self, q, k, v, softmax_scale: float = 0.0, stream=None):
         block_sparse_attn(self.p, q, k, v, self.counts, self.indices, softmax_scale, self.out, self.lse,

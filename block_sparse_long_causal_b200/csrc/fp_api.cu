@@ -209,18 +209,12 @@ fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float
   return cuda_status(fp::launch_pool(a, grid, static_cast<cudaStream_t>(stream)), "pool launch");
 }
 
-fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
-                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
-  fp_status st = check_problem(p);
-  if (st != FP_OK) return st;
-  if (!q_pool || !k_pool || !counts || !indices)
-    return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, counts and indices must be non-NULL");
-  if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
-  if (!std::isfinite(tau)) return fail(FP_ERR_INVALID_ARG, "tau must be finite");
-  if (p->total_blocks == 0) return FP_OK;
+namespace {
+fp::SearchParams search_params(const fp_problem* p, float tau, const float* k_pool, int32_t* counts,
+                               int32_t* indices, int32_t* dev_status) {
   fp::SearchParams a;
+  memset(&a, 0, sizeof a);
   a.seq = seq_info(p);
-  a.q_pool = q_pool;
   a.k_pool = k_pool;
   a.hq = p->num_q_heads;
   a.hkv = p->num_kv_heads;
@@ -235,7 +229,30 @@ fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float*
   a.indices = indices;
   a.index_elems = p->index_elems;
   a.dev_status = dev_status;
+  return a;
+}
+}  // namespace
+
+fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
+                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!q_pool || !k_pool || !counts || !indices)
+    return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, counts and indices must be non-NULL");
+  if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
+  if (!std::isfinite(tau)) return fail(FP_ERR_INVALID_ARG, "tau must be finite");
+  if (p->total_blocks == 0) return FP_OK;
+  fp::SearchParams a = search_params(p, tau, k_pool, counts, indices, dev_status);
+  a.q_pool = q_pool;
   return cuda_status(fp::launch_search(a, static_cast<cudaStream_t>(stream)), "search launch");
+}
+
+fp_status fp_block_pool_search(const fp_problem* p, const void* q, const void* k, float tau, float* q_pool,
+                               float* k_pool, int32_t* counts, int32_t* indices, int32_t* dev_status,
+                               void* stream) {
+  fp_status st = fp_block_pool(p, q, k, q_pool, k_pool, stream);
+  if (st != FP_OK) return st;
+  return fp_block_search(p, q_pool, k_pool, tau, counts, indices, dev_status, stream);
 }
 
 fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,

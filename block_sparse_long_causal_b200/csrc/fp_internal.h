@@ -31,7 +31,7 @@ struct PoolParams {
 
 struct SearchParams {
   SeqInfo seq;
-  const float* q_pool;
+  const float* q_pool;        // pooled queries [NB, Hq, d]
   const float* k_pool;
   int32_t hq, hkv, group;     // group = Hq / Hkv
   int32_t rows_blocks;        // query blocks per CTA tile (TI)

@@ -15,6 +15,8 @@
 // loads (the dominant bytes); the search kernel reads the small pooled tensors (L2 resident),
 // keeps the pooled scores in registers (never materialised), reduces the row max with warp
 // shuffles and writes the lists with ballot/popc compaction.
+#include <cuda_bf16.h>
+
 #include "fp_internal.h"
 #include "fp_seq.cuh"
 
@@ -89,16 +91,22 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
 // ---------------------------------------------------------------------------------- search ----
 // CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows (q-head, block) that
 // all share the pooled keys of kv-head g (GQA). Row r: head offset r % G, block offset r / G.
-// Pooled keys stream through shared memory in chunks of 64 blocks, double buffered with cp.async
-// (16-byte global->shared copies in flight while the previous chunk is scored). Warp w scores key
-// blocks 8w..8w+7 of a chunk (broadcast shared reads) against rows 2l, 2l+1 of lane l (pooled
-// queries transposed in shared memory): per 4 steps of d, 8 broadcast and 4 lane-private loads
-// feed 64 FMAs, so the loop is bound by the FMA pipe.
-// Pass 1: row max m_i and row min of s_ij over j <= i (scores stay in registers).
-// If min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
-// same decision the per-block test would take) and the row is written as 0..i directly.
-// Otherwise pass 2 recomputes the scores, stages them in shared memory, and one warp per 8 rows
-// emits the kept blocks in ascending order with ballot/popc compaction.
+// Scores, row max / min, threshold and emission happen in this one kernel; the block-score matrix
+// is never written to memory. Two CTAs fit on an SM.
+// Pooled keys stream through shared memory in chunks of 64 blocks (cp.async, next chunk in flight).
+// Warp w scores key blocks 8w..8w+7 of a chunk (broadcast shared reads) against rows 2l, 2l+1 of
+// lane l (pooled queries transposed in shared memory).
+// Pass 0 (tensor cores): approximate row max / min of the pooled scores with mma.sync bf16 on a
+// two-term split of the fp32 operands (x = hi + lo; q.k ~ qh.kh + qh.kl + ql.kh) and a rigorous
+// per-row error bound eps_i = 2^-14 * |q_i| * max_j |k_j| / sqrt(d) (the dropped terms and the
+// fp32 accumulation are below 2^-15 * sum_d |q_d k_d| <= 2^-15 * |q| |k|). A row is certainly
+// all-kept when (min - max) - 2 eps >= ln(tau); it is then written as 0..i.
+// If any row of the tile is not certain, the tile takes the exact fp32 path:
+// Pass 1: exact row max m_i and row min of s_ij over j <= i (scores stay in registers); if
+// min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
+// decision the per-block test would take) and the row is written as 0..i.
+// Pass 2: recompute the exact scores, stage them in shared memory, and one warp per 8 rows emits
+// the kept blocks in ascending order with ballot/popc compaction.
 constexpr int kSearchThreads = 256;
 constexpr int kSearchWarps = kSearchThreads / 32;
 constexpr int kSearchRows = 64;
@@ -106,16 +114,28 @@ constexpr int kKChunk = 64;                  // key blocks per chunk (8 per warp
 constexpr int kQTStride = kSearchRows + 4;   // transposed pooled-query row stride (floats)
 constexpr int kKStride = kHeadDim + 4;       // pooled-key row stride (floats), 16-byte aligned
 
+// Shared memory: fixed part, then the sequence tables sized for this launch's sequence count.
+// k[1] doubles as the pass-2 score tile (see the assert).
 struct SearchSmem {
   float k[2][kKChunk][kKStride];             // pooled keys, natural layout, two buffers
   float qT[kHeadDim][kQTStride];             // pooled queries, [d][row]
   float red[2][kSearchWarps][kSearchRows];   // per-warp row max / min
-  float sc[kSearchRows][kKChunk + 1];        // chunk scores for the emission pass
-  int cu[kMaxSeqs + 1], cb[kMaxSeqs + 1], ct[kMaxSeqs + 1];
-  long long ib[kMaxSeqs + 1];
+  float qnorm[kSearchRows];                  // |q_row| (pass 0 error bound)
+  int kmax_bits;                             // max |k_j| of the tile's keys, as float bits
   int ok;
   int need_pass2;
+  int need_exact;
 };
+// Pass-0 operand views: split bf16 [hi/lo][row][kBfStride] in the qT region (queries) and in the
+// key region (keys); the padded stride keeps the 32-bit fragment loads conflict free.
+constexpr int kBfStride = kHeadDim + 8;
+static_assert(2 * kSearchRows * kBfStride * 2 <= (int)sizeof(float) * kHeadDim * kQTStride, "query split view");
+static_assert(2 * kKChunk * kBfStride * 2 <= (int)sizeof(float) * 2 * kKChunk * kKStride, "key split view");
+static_assert(kSearchRows * (kKChunk + 1) <= kKChunk * kKStride, "score tile must fit in one key buffer");
+
+__host__ __device__ inline size_t search_smem_bytes(int num_seqs) {
+  return sizeof(SearchSmem) + (size_t)(num_seqs + 1) * (3 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
+}
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
   const uint32_t d = smem_u32(dst);
@@ -161,14 +181,118 @@ __device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int buf, int 
   }
 }
 
-__global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchParams p) {
+__device__ __forceinline__ uint32_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+// Split 4 fp32 values into bf16 hi and lo (x - hi) and store them at hi_dst / lo_dst (8 bytes each).
+__device__ __forceinline__ void split_store4(uint16_t* hi_dst, uint16_t* lo_dst, float4 v) {
+  const float x[4] = {v.x, v.y, v.z, v.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    h[e] = bf16_bits(x[e]);
+    l[e] = bf16_bits(x[e] - __uint_as_float(h[e] << 16));
+  }
+  *reinterpret_cast<uint2*>(hi_dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+  *reinterpret_cast<uint2*>(lo_dst) = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+}
+
+// 64 rows x 128 fp32 (rows via row_ptr) -> split bf16 view; optional per-row norms.
+// Warp w handles rows w, w + 8, ...; lane l the 4 columns 4l..4l+3.
+template <typename RowPtr>
+__device__ __forceinline__ void load_split_rows(uint16_t* view, RowPtr row_ptr, float* norms, int* max_bits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kPer = kSearchRows / kSearchWarps;
+  float4 vv[kPer];  // all loads in flight before any use (L2 latency paid once)
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const float* src = row_ptr(warp + q * kSearchWarps);
+    vv[q] = src ? reinterpret_cast<const float4*>(src)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int r = warp + q * kSearchWarps;
+    const float4 v = vv[q];
+    split_store4(view + r * kBfStride + 4 * lane, view + (kSearchRows + r) * kBfStride + 4 * lane, v);
+    float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) {
+      const float nrm = sqrtf(ss);
+      if (norms) norms[r] = nrm;
+      if (max_bits) atomicMax(max_bits, __float_as_int(nrm));
+    }
+  }
+}
+
+// Pass-0 key staging: fp32 chunk [64 rows][128] (unpadded) in the upper half of the key region, filled
+// by cp.async while the previous chunk's MMAs run.
+constexpr int kStageOffBytes = 2 * kKChunk * kBfStride * 2;
+static_assert(kStageOffBytes + kKChunk * kHeadDim * 4 <= (int)sizeof(float) * 2 * kKChunk * kKStride, "staging");
+
+__device__ __forceinline__ void issue_stage_chunk(float* stage, const float* kp, int gb0, int g, int hkv, int j0,
+                                                  int jmax) {
+  for (int e = threadIdx.x; e < kKChunk * (kHeadDim / 4); e += kSearchThreads) {
+    const int jr = e / (kHeadDim / 4), c4 = e % (kHeadDim / 4);
+    const int j = min(j0 + jr, jmax);
+    cp_async16(stage + jr * kHeadDim + 4 * c4, kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim + 4 * c4,
+               j0 + jr <= jmax);
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Pass-0 scores of one 64-block chunk: warp w covers rows 16(w%4).. and key blocks 32(w/4)..;
+// acc[nt][e]: rows r0+g (e = 0,1) and r0+g+8 (e = 2,3), key blocks n0+8nt+2t+(e&1).
+__device__ __forceinline__ void chunk_scores_tc(const uint16_t* qv, const uint16_t* kv, int warp, int lane,
+                                                float (&acc)[4][4]) {
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  auto w32 = [](const uint16_t* base, int row, int col) {
+    return *reinterpret_cast<const uint32_t*>(base + row * kBfStride + col);
+  };
+  const uint16_t* qh = qv;
+  const uint16_t* ql = qv + kSearchRows * kBfStride;
+  const uint16_t* kh = kv;
+  const uint16_t* kl = kv + kKChunk * kBfStride;
+#pragma unroll 2
+  for (int kk = 0; kk < kHeadDim; kk += 16) {
+    const int c0 = kk + 2 * t;
+    const uint32_t ah[4] = {w32(qh, r0 + g, c0), w32(qh, r0 + g + 8, c0), w32(qh, r0 + g, c0 + 8), w32(qh, r0 + g + 8, c0 + 8)};
+    const uint32_t al[4] = {w32(ql, r0 + g, c0), w32(ql, r0 + g + 8, c0), w32(ql, r0 + g, c0 + 8), w32(ql, r0 + g + 8, c0 + 8)};
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int n = n0 + 8 * nt + g;
+      const uint32_t bh0 = w32(kh, n, c0), bh1 = w32(kh, n, c0 + 8);
+      const uint32_t bl0 = w32(kl, n, c0), bl1 = w32(kl, n, c0 + 8);
+      mma_bf16_16816(acc[nt], ah, bh0, bh1);
+      mma_bf16_16816(acc[nt], ah, bl0, bl1);
+      mma_bf16_16816(acc[nt], al, bh0, bh1);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchParams p) {
   extern __shared__ __align__(16) unsigned char search_smem_raw[];
   SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
-  if (!build_seq_tables(p.seq, sm.cu, sm.cb, sm.ct, sm.ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
+  const int S = p.seq.num_seqs;
+  int* t_cu = reinterpret_cast<int*>(search_smem_raw + sizeof(SearchSmem));
+  int* t_cb = t_cu + (S + 1);
+  int* t_ct = t_cb + (S + 1);
+  long long* t_ib = reinterpret_cast<long long*>(((uintptr_t)(t_ct + (S + 1)) + 7) & ~(uintptr_t)7);
+  if (!build_seq_tables(p.seq, t_cu, t_cb, t_ct, t_ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
                         p.dev_status))
     return;
-  const int S = p.seq.num_seqs;
-  if (sm.ib[S] != p.index_elems) {
+  if (t_ib[S] != p.index_elems) {
     if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
     return;
   }
@@ -177,98 +301,181 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
   const int NB = p.seq.total_blocks;
   const unsigned lt_mask = (1u << lane) - 1u;
 
-  const int num_tiles = sm.ct[S];
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-    const int s = find_seq(sm.ct, S, tile);
-    const int local = tile - sm.ct[s];
-    const int nb = sm.cb[s + 1] - sm.cb[s];
+  const int num_tiles = t_ct[S];
+  // boustrophedon over the grid: tiles are heaviest first, so alternating direction per round
+  // balances the per-CTA work without a work queue
+  for (int kr = 0;; ++kr) {
+    const int tile = kr * gridDim.x + ((kr & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+    if (tile >= num_tiles) break;
+    const int s = find_seq(t_ct, S, tile);
+    const int local = tile - t_ct[s];
+    const int nb = t_cb[s + 1] - t_cb[s];
     const int ntiles = (nb + TI - 1) / TI;
     const int it = ntiles - 1 - local / p.hkv;  // heavy (late) query blocks first
     const int g = local % p.hkv;
     const int i0 = it * TI;
     const int i_last = min(i0 + TI, nb) - 1;
-    const int gb0 = sm.cb[s];
+    const int gb0 = t_cb[s];
     const int nchunks = i_last / kKChunk + 1;
 
     __syncthreads();  // previous tile done with shared memory
-    if (!p.keep_all) issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, 0, i_last);
-    for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
-      const int r = e % kSearchRows, d4 = e / kSearchRows;
-      const int i = i0 + r / G, h = g * G + r % G;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < TI * G && i <= i_last)
-        v = reinterpret_cast<const float4*>(p.q_pool + ((long long)(gb0 + i) * p.hq + h) * kHeadDim)[d4];
-      sm.qT[4 * d4 + 0][r] = v.x;
-      sm.qT[4 * d4 + 1][r] = v.y;
-      sm.qT[4 * d4 + 2][r] = v.z;
-      sm.qT[4 * d4 + 3][r] = v.w;
+    const float* q_src = p.q_pool;  // pooled queries of the tile (global, L2 resident)
+    auto q_row = [&](int r) -> const float* {
+      const int i = i0 + r / G;
+      return (r < TI * G && i <= i_last) ? q_src + ((long long)(gb0 + i) * p.hq + g * G + r % G) * kHeadDim : nullptr;
+    };
+    if (threadIdx.x == 0) {
+      sm.need_pass2 = 0;
+      sm.need_exact = 0;
+      sm.kmax_bits = 0;
     }
-    if (threadIdx.x == 0) sm.need_pass2 = 0;
-
-    // scoring rows of this lane
-    int li[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = 2 * lane + e;
-      li[e] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
-    }
-    float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
-
-    if (!p.keep_all) {
-      // ---- pass 1: row max / min of the pooled scores
-      for (int c = 0; c < nchunks; ++c) {
-        const int j0 = c * kKChunk;
-        if (c + 1 < nchunks) {
-          __syncthreads();  // buffer (c+1)&1 no longer read
-          issue_k_chunk(sm, (c + 1) & 1, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
-          cp_async_wait_all_but_one();
-        } else {
-          cp_async_wait_all();
-        }
-        __syncthreads();
-        float acc[2][8];
-        chunk_scores(sm, c & 1, warp, lane, acc);
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            if (j0 + 8 * warp + b <= li[e]) {
-              const float sc = acc[e][b] * p.inv_sqrt_d;
-              mx[e] = fmaxf(mx[e], sc);
-              mn[e] = fminf(mn[e], sc);
-            }
-          }
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        sm.red[0][warp][2 * lane + e] = mx[e];
-        sm.red[1][warp][2 * lane + e] = mn[e];
-      }
-    }
-    __syncthreads();
 
     // emission rows: warp w emits rows 8w..8w+7
     int row_i[8], row_h[8];
-    float rmx[8];
-    bool all_keep[8];
-    bool warp_needs = false;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int rr = warp * 8 + r;
       row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
       row_h[r] = g * G + rr % G;
-      float a = -INFINITY, b = INFINITY;
-      if (!p.keep_all) {
+    }
+    bool all_keep[8];
+    float rmx[8];
 #pragma unroll
-        for (int w = 0; w < kSearchWarps; ++w) {
-          a = fmaxf(a, sm.red[0][w][rr]);
-          b = fminf(b, sm.red[1][w][rr]);
+    for (int r = 0; r < 8; ++r) { all_keep[r] = true; rmx[r] = 0.f; }
+
+    if (!p.keep_all) {
+      // ---- pass 0: approximate max / min on tensor cores, with a rigorous error bound
+      uint16_t* qv = reinterpret_cast<uint16_t*>(&sm.qT[0][0]);
+      uint16_t* kvw = reinterpret_cast<uint16_t*>(&sm.k[0][0][0]);
+      __syncthreads();
+      load_split_rows(qv, q_row, sm.qnorm, nullptr);
+      const int g4 = lane >> 2, t4 = lane & 3;
+      const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+      int ri[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = r0 + g4 + 8 * h2;
+        ri[h2] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+      }
+      float am[2] = {-INFINITY, -INFINITY}, an[2] = {INFINITY, INFINITY};
+      float* stage = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(kvw) + kStageOffBytes);
+      issue_stage_chunk(stage, p.k_pool, gb0, g, p.hkv, 0, i_last);
+      for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
+        cp_async_wait_all();
+        __syncthreads();  // staged chunk visible; previous chunk's MMAs done with the split view
+        load_split_rows(kvw, [&](int jr) -> const float* { return stage + jr * kHeadDim; }, nullptr,
+                        &sm.kmax_bits);
+        __syncthreads();  // split view ready; staging free
+        if (j0 + kKChunk <= i_last) issue_stage_chunk(stage, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
+        float acc[4][4];
+        chunk_scores_tc(qv, kvw, warp, lane, acc);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j0 + n0 + 8 * nt + 2 * t4 + (e & 1);
+            const int h2 = e >> 1;
+            if (j <= ri[h2]) {
+              const float sc = acc[nt][e] * p.inv_sqrt_d;
+              am[h2] = fmaxf(am[h2], sc);
+              an[h2] = fminf(an[h2], sc);
+            }
+          }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          am[h2] = fmaxf(am[h2], __shfl_xor_sync(0xffffffffu, am[h2], o));
+          an[h2] = fminf(an[h2], __shfl_xor_sync(0xffffffffu, an[h2], o));
+        }
+        if (t4 == 0) {
+          sm.red[0][warp >> 2][r0 + g4 + 8 * h2] = am[h2];
+          sm.red[1][warp >> 2][r0 + g4 + 8 * h2] = an[h2];
         }
       }
-      rmx[r] = a;
-      all_keep[r] = p.keep_all || (b - a >= p.log_tau);
-      if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
+      __syncthreads();
+      const float kmax = __int_as_float(sm.kmax_bits);
+      bool uncertain = false;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int rr = warp * 8 + r;
+        const float a = fmaxf(sm.red[0][0][rr], sm.red[0][1][rr]);
+        const float b = fminf(sm.red[1][0][rr], sm.red[1][1][rr]);
+        const float eps = 6.103515625e-05f * sm.qnorm[rr] * kmax * p.inv_sqrt_d;  // 2^-14 |q| max|k| / sqrt(d)
+        if (row_i[r] >= 0 && !((b - a) - 2.f * eps >= p.log_tau)) uncertain = true;
+      }
+      if (uncertain && lane == 0) atomicOr(&sm.need_exact, 1);
+      __syncthreads();
+
+      if (sm.need_exact) {
+        // ---- exact fp32 path for this tile
+        for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
+          const int r = e % kSearchRows, d4 = e / kSearchRows;
+          const float* src = q_row(r);
+          const float4 v = src ? reinterpret_cast<const float4*>(src)[d4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          sm.qT[4 * d4 + 0][r] = v.x;
+          sm.qT[4 * d4 + 1][r] = v.y;
+          sm.qT[4 * d4 + 2][r] = v.z;
+          sm.qT[4 * d4 + 3][r] = v.w;
+        }
+        issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, 0, i_last);
+        // scoring rows of this lane
+        int li[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = 2 * lane + e;
+          li[e] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+        }
+        float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
+        // ---- pass 1: exact row max / min of the pooled scores
+        for (int c = 0; c < nchunks; ++c) {
+          const int j0 = c * kKChunk;
+          if (c + 1 < nchunks) {
+            __syncthreads();  // buffer (c+1)&1 no longer read
+            issue_k_chunk(sm, (c + 1) & 1, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
+            cp_async_wait_all_but_one();
+          } else {
+            cp_async_wait_all();
+          }
+          __syncthreads();
+          float acc[2][8];
+          chunk_scores(sm, c & 1, warp, lane, acc);
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              if (j0 + 8 * warp + b <= li[e]) {
+                const float sc = acc[e][b] * p.inv_sqrt_d;
+                mx[e] = fmaxf(mx[e], sc);
+                mn[e] = fminf(mn[e], sc);
+              }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          sm.red[0][warp][2 * lane + e] = mx[e];
+          sm.red[1][warp][2 * lane + e] = mn[e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int rr = warp * 8 + r;
+          float a = -INFINITY, b = INFINITY;
+#pragma unroll
+          for (int w = 0; w < kSearchWarps; ++w) {
+            a = fmaxf(a, sm.red[0][w][rr]);
+            b = fminf(b, sm.red[1][w][rr]);
+          }
+          rmx[r] = a;
+          all_keep[r] = (b - a >= p.log_tau);
+        }
+      }
     }
+    bool warp_needs = false;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
     const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
                               max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
     if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
@@ -276,7 +483,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
     for (int r = 0; r < 8; ++r) {
       if (row_i[r] < 0 || !all_keep[r]) continue;
       const int i = row_i[r];
-      int32_t* dst = p.indices + list_row(sm.cb, sm.ib, s, row_h[r], i);
+      int32_t* dst = p.indices + list_row(t_cb, t_ib, s, row_h[r], i);
       for (int j = lane; j <= i; j += 32) dst[j] = j;
       if (lane == 0) p.counts[(long long)row_h[r] * NB + gb0 + i] = i + 1;
     }
@@ -284,12 +491,13 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
     if (!sm.need_pass2) continue;
 
     // ---- pass 2: recompute the scores and emit kept blocks in ascending order
+    float(*sc)[kKChunk + 1] = reinterpret_cast<float(*)[kKChunk + 1]>(&sm.k[1][0][0]);
     int cnt[8];
     int64_t base[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       cnt[r] = 0;
-      base[r] = (row_i[r] >= 0) ? list_row(sm.cb, sm.ib, s, row_h[r], row_i[r]) : 0;
+      base[r] = (row_i[r] >= 0) ? list_row(t_cb, t_ib, s, row_h[r], row_i[r]) : 0;
     }
     for (int c = 0; c < nchunks; ++c) {
       const int j0 = c * kKChunk;
@@ -302,7 +510,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
 #pragma unroll
       for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) sm.sc[2 * lane + e][8 * warp + b] = acc[e][b] * p.inv_sqrt_d;
+        for (int b = 0; b < 8; ++b) sc[2 * lane + e][8 * warp + b] = acc[e][b] * p.inv_sqrt_d;
       __syncthreads();
       if (!warp_needs || j0 > warp_imax) continue;
 #pragma unroll
@@ -311,8 +519,8 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
 #pragma unroll
         for (int h2 = 0; h2 < kKChunk; h2 += 32) {
           const int j = j0 + h2 + lane;
-          const float sc = sm.sc[warp * 8 + r][h2 + lane];
-          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || sc - rmx[r] >= p.log_tau);
+          const float v = sc[warp * 8 + r][h2 + lane];
+          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || v - rmx[r] >= p.log_tau);
           const unsigned bal = __ballot_sync(0xffffffffu, keep);
           if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
           cnt[r] += __popc(bal);
@@ -329,16 +537,18 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_kernel(const SearchP
 
 cudaError_t launch_search(const SearchParams& p, cudaStream_t st) {
   static bool attr_done = false;
-  const int smem = (int)sizeof(SearchSmem);
+  const int smem = (int)search_smem_bytes(p.seq.num_seqs);
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(search_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(search_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)search_smem_bytes(kMaxSeqs));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  const int cap = 2 * sms;
+  const int grid = p.num_tiles < cap ? p.num_tiles : cap;
   if (grid <= 0) return cudaSuccess;
   search_kernel<<<grid, kSearchThreads, smem, st>>>(p);
   return cudaGetLastError();

@@ -107,6 +107,14 @@ FP_API fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k
 FP_API fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
                           int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream);
 
+/* Steps 1 + 2 in one call: fp_block_pool followed by fp_block_search on the same stream (two
+ * launches: Q and K are streamed once by the pool kernel at HBM bandwidth; the search kernel
+ * then computes the block scores, the threshold and the lists without materialising scores).
+ * q_pool and k_pool are required outputs (the pooled tensors). */
+FP_API fp_status fp_block_pool_search(const fp_problem* p, const void* q, const void* k, float tau, float* q_pool,
+                               float* k_pool, int32_t* counts, int32_t* indices, int32_t* dev_status,
+                               void* stream);
+
 /* Step 3 -- block-sparse causal attention over the listed blocks (online softmax, bf16 in,
  * fp32 accumulate, bf16 out). counts/indices as written by fp_block_search (any ascending lists
  * of local block ids <= i are accepted; out-of-range entries are skipped and flagged).

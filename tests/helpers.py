@@ -97,15 +97,18 @@ def compare_lists(g_counts, g_idx, o_counts, o_idx, o_band, cu, B, hq):
     return int(diff.sum()), int(mo.sum())
 
 
-def gpu_prefill(x, hq, hkv, B, tau, dense=False, with_lse=True, check_status=True):
-    """Run pool + search + sparse (or dense) attention through the C ABI on cuda:0."""
+def gpu_prefill(x, hq, hkv, B, tau, dense=False, with_lse=True, check_status=True, fused=True):
+    """Run pool + search + sparse (or dense) attention through the C ABI on cuda:0.
+
+    fused=True uses the one-call fp_block_pool_search; fused=False calls fp_block_pool and
+    fp_block_search separately."""
     import torch
     import block_sparse_long_causal_b200 as fp
     cu = x["cu_seqlens"]
     p = fp.problem(cu, hq, hkv, 128, B)
     sp = fp.SparsePrefill(p, with_lse=with_lse)
     q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
-    sp.search(q, k, tau)
+    sp.search(q, k, tau, fused=fused)
     if dense:
         sp.dense(q, k, v)
     else:

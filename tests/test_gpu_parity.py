@@ -28,8 +28,8 @@ def _oracle_lists(x, B, tau):
     return qb, kb, oracle.search(qb, kb, cu, B, tau)
 
 
-def _check_case(x, hq, hkv, B, tau, rows=None, rel_max=2e-2):
-    res = gpu_prefill(x, hq, hkv, B, tau)
+def _check_case(x, hq, hkv, B, tau, rows=None, rel_max=2e-2, fused=True):
+    res = gpu_prefill(x, hq, hkv, B, tau, fused=fused)
     qb, kb, (oc, oi, band) = _oracle_lists(x, B, tau)
     np.testing.assert_allclose(res["q_pool"], qb, rtol=0, atol=5e-5)
     np.testing.assert_allclose(res["k_pool"], kb, rtol=0, atol=5e-5)
@@ -70,6 +70,15 @@ def test_mha4_L2048_B64(tau):
     w = synth.WORKLOADS["mha4-L2048-B64"]
     x = synth.make_inputs(w)
     _check_case(x, w.hq, w.hkv, w.block, tau)
+
+
+@pytest.mark.parametrize("case", [SMALL[1], SMALL[4], SMALL[6], SMALL[8]],
+                         ids=["L300", "varlen", "B64-varlen", "G3"])
+def test_unfused_pool_then_search(case):
+    """fp_block_pool and fp_block_search called separately (the two steps) against the oracle."""
+    lens, hq, hkv, B, tau, scale = case
+    x = synth.random_inputs(lens, hq, hkv, 128, seed=sum(lens) + hq, scale=scale)
+    _check_case(x, hq, hkv, B, tau, fused=False)
 
 
 def test_dense_matches_oracle_dense():
