@@ -11,6 +11,7 @@ Entry points mirror the C ABI in include/fp.h:
     block_pool_search(...)  -> fp_block_pool_search (steps 1 + 2 fused)
     block_sparse_attn(...)  -> fp_block_sparse_attn
     dense_attn(...)         -> fp_dense_attn
+    sparse_prefill(...)     -> fp_sparse_prefill (all three steps, caller workspace)
     validate_lists(...)     -> fp_validate_lists
 and SparsePrefill bundles the three steps with caller-side buffers.
 """
@@ -29,7 +30,7 @@ FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 
 FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
 FP_MAX_SEQS = 1024
 EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_pool_search", "fp_block_sparse_attn",
-            "fp_dense_attn",
+            "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill",
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version")
 
 
@@ -61,6 +62,8 @@ def _load():
         "fp_dense_attn": [P, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_validate_lists": [P, vp, vp, vp, vp],
         "fp_selftest_exp2": [vp, vp, vp, C.c_int64, vp],
+        "fp_sparse_prefill_workspace": [P, C.POINTER(C.c_int64)],
+        "fp_sparse_prefill": [P, vp, vp, vp, f32, f32, vp, C.c_int64, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -159,6 +162,19 @@ def dense_attn(p: Problem, q, k, v, softmax_scale: float, out, lse=None, dev_sta
 
 def validate_lists(p: Problem, counts, indices, dev_status, stream=None):
     _check(_lib.fp_validate_lists(p.ref, _ptr(counts), _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
+def sparse_prefill_workspace(p: Problem) -> int:
+    n = C.c_int64(0)
+    _check(_lib.fp_sparse_prefill_workspace(p.ref, C.byref(n)))
+    return int(n.value)
+
+
+def sparse_prefill(p: Problem, q, k, v, tau: float, softmax_scale: float, workspace, out, lse=None, dev_status=None,
+                   stream=None):
+    _check(_lib.fp_sparse_prefill(p.ref, _ptr(q), _ptr(k), _ptr(v), float(tau), float(softmax_scale),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
+                                  _ptr(dev_status), _stream(stream)))
 
 
 def selftest_exp2(x, y_poly, y_mufu, stream=None):

@@ -266,6 +266,52 @@ fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const
   return attn_common(p, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
 }
 
+namespace {
+struct WorkspaceLayout {
+  int64_t q_pool, k_pool, counts, indices, total;  // byte offsets and total size
+};
+int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
+WorkspaceLayout workspace_layout(const fp_problem* p) {
+  WorkspaceLayout w;
+  const int64_t nb = p->total_blocks, d = p->head_dim;
+  w.q_pool = 0;
+  w.k_pool = align256(w.q_pool + nb * p->num_q_heads * d * 4);
+  w.counts = align256(w.k_pool + nb * p->num_kv_heads * d * 4);
+  w.indices = align256(w.counts + (int64_t)p->num_q_heads * nb * 4);
+  w.total = align256(w.indices + p->index_elems * 4);
+  return w;
+}
+}  // namespace
+
+fp_status fp_sparse_prefill_workspace(const fp_problem* p, int64_t* bytes) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!bytes) return fail(FP_ERR_INVALID_ARG, "bytes must be non-NULL");
+  *bytes = workspace_layout(p).total;
+  return FP_OK;
+}
+
+fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, const void* v, float tau,
+                            float softmax_scale, void* workspace, int64_t workspace_bytes, void* out, float* lse,
+                            int32_t* dev_status, void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  const WorkspaceLayout w = workspace_layout(p);
+  if (!workspace) return fail(FP_ERR_INVALID_ARG, "workspace must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(FP_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld bytes needed",
+                (long long)workspace_bytes, (long long)w.total);
+  char* base = static_cast<char*>(workspace);
+  float* q_pool = reinterpret_cast<float*>(base + w.q_pool);
+  float* k_pool = reinterpret_cast<float*>(base + w.k_pool);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + w.counts);
+  int32_t* indices = reinterpret_cast<int32_t*>(base + w.indices);
+  if ((st = fp_block_pool(p, q, k, q_pool, k_pool, stream)) != FP_OK) return st;
+  if ((st = fp_block_search(p, q_pool, k_pool, tau, counts, indices, dev_status, stream)) != FP_OK) return st;
+  return fp_block_sparse_attn(p, q, k, v, counts, indices, softmax_scale, out, lse, dev_status, stream);
+}
+
 fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices, int32_t* dev_status,
                             void* stream) {
   fp_status st = check_problem(p);

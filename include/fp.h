@@ -129,6 +129,19 @@ FP_API fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const 
 FP_API fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
                         void* out, float* lse, int32_t* dev_status, void* stream);
 
+/* Bytes of workspace fp_sparse_prefill needs for this problem: the pooled Q and K, the counts and
+ * the index lists, each 256-byte aligned. */
+FP_API fp_status fp_sparse_prefill_workspace(const fp_problem* p, int64_t* bytes);
+
+/* The whole sparse prefill in one call (FlashPrefill: block pooling, max-based block search and
+ * block-sparse attention): fp_block_pool, fp_block_search and fp_block_sparse_attn on `stream`,
+ * with the intermediate tensors in `workspace` (device, 256-byte aligned, at least
+ * fp_sparse_prefill_workspace bytes; its contents are scratch and are overwritten).
+ * out / lse / softmax_scale / dev_status as for fp_block_sparse_attn. */
+FP_API fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, const void* v, float tau,
+                            float softmax_scale, void* workspace, int64_t workspace_bytes, void* out, float* lse,
+                            int32_t* dev_status, void* stream);
+
 /* Device-side check of index lists: every row's count in [1, i+1], entries ascending, in [0, i],
  * first entry 0 and last entry i. Violations OR FP_DEV_BAD_LIST into dev_status (required). */
 FP_API fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices,

@@ -103,3 +103,21 @@ def test_binding_raises_fp_error():
     with pytest.raises(fp.FpError):
         fp.Problem(np.array([0, 10], np.int32), __import__("torch").zeros(2, dtype=__import__("torch").int32),
                    4, 2, 64, 128)
+
+
+def test_sparse_prefill_workspace_and_argument_checks():
+    st, p = _prob((0, 300, 301, 700), hq=4, hkv=2, B=128)
+    assert st == fp.FP_OK
+    n = C.c_int64(0)
+    assert fp._lib.fp_sparse_prefill_workspace(C.byref(p), C.byref(n)) == fp.FP_OK
+    nb = 3 + 1 + 4
+    need = 0
+    for nbytes in (nb * 4 * 128 * 4, nb * 2 * 128 * 4, 4 * nb * 4, p.index_elems * 4):
+        need += (nbytes + 255) // 256 * 256
+    assert n.value == need
+    ok, null = C.c_void_p(4096), None
+    args = lambda ws, nbytes: (C.byref(p), ok, ok, ok, C.c_float(0.1), C.c_float(0), ws, nbytes, ok, null, null, null)
+    assert fp._lib.fp_sparse_prefill(*args(null, n.value)) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_sparse_prefill(*args(C.c_void_p(4096 + 16), n.value)) == fp.FP_ERR_INVALID_ARG  # not 256-aligned
+    assert fp._lib.fp_sparse_prefill(*args(ok, n.value - 1)) == fp.FP_ERR_INVALID_ARG
+    assert "workspace" in _err()

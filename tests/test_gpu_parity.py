@@ -131,3 +131,23 @@ def test_exp2_polynomial_error_bound():
     torch.cuda.synchronize()
     v = yp2.cpu().numpy()
     assert (v >= 0).all() and (v <= 2.0 ** -125).all()
+
+
+def test_one_call_sparse_prefill_matches_the_three_calls():
+    import torch
+    import block_sparse_long_causal_b200 as fp
+    from helpers import bf16_to_np, to_dev
+    w = synth.WORKLOADS["llama3-8b-L32768"]
+    x = synth.make_inputs(w.with_lens([3000, 129, 1800]))
+    ref = gpu_prefill(x, w.hq, w.hkv, w.block, 0.9)
+    p = fp.problem(x["cu_seqlens"], w.hq, w.hkv, 128, w.block)
+    ws = torch.empty(fp.sparse_prefill_workspace(p), dtype=torch.uint8, device="cuda")
+    out = torch.empty((p.total_tokens, w.hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.hq, p.total_tokens), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    fp.sparse_prefill(p, q, k, v, 0.9, 0.0, ws, out, lse, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(bf16_to_np(out), ref["out"])
+    np.testing.assert_array_equal(lse.cpu().numpy(), ref["lse"])
