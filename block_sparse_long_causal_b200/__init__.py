@@ -29,8 +29,9 @@ LIB_PATH = os.path.join(_HERE, "libfp.so")
 FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 1, 2, 3, 4
 FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
 FP_MAX_SEQS = 1024
+FP_NOALLOC_MAX_BYTES = 64 << 20
 EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_pool_search", "fp_block_sparse_attn",
-            "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill",
+            "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill", "fp_sparse_prefill_noalloc",
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version")
 
 
@@ -64,6 +65,7 @@ def _load():
         "fp_selftest_exp2": [vp, vp, vp, C.c_int64, vp],
         "fp_sparse_prefill_workspace": [P, C.POINTER(C.c_int64)],
         "fp_sparse_prefill": [P, vp, vp, vp, f32, f32, vp, C.c_int64, vp, vp, vp, vp],
+        "fp_sparse_prefill_noalloc": [P, vp, vp, vp, f32, f32, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -175,6 +177,13 @@ def sparse_prefill(p: Problem, q, k, v, tau: float, softmax_scale: float, worksp
     _check(_lib.fp_sparse_prefill(p.ref, _ptr(q), _ptr(k), _ptr(v), float(tau), float(softmax_scale),
                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
                                   _ptr(dev_status), _stream(stream)))
+
+
+def sparse_prefill_noalloc(p: Problem, q, k, v, tau: float, softmax_scale: float, out, lse=None, dev_status=None,
+                           stream=None):
+    """fp_sparse_prefill for callers that cannot allocate: intermediates in the library's static array."""
+    _check(_lib.fp_sparse_prefill_noalloc(p.ref, _ptr(q), _ptr(k), _ptr(v), float(tau), float(softmax_scale),
+                                          _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
 
 
 def selftest_exp2(x, y_poly, y_mufu, stream=None):

@@ -149,6 +149,16 @@ fp_status attn_common(const fp_problem* p, const void* q, const void* k, const v
 
 }  // namespace
 
+namespace fp {
+fp_status set_error(fp_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+}  // namespace fp
+
 extern "C" {
 
 fp_status fp_problem_init(fp_problem* p, const int32_t* host_cu, int32_t num_seqs, const int32_t* dev_cu,

@@ -77,6 +77,9 @@ constexpr int kMaxSeqs = FP_MAX_SEQS;
 constexpr int kHeadDim = 128;
 constexpr int kTileM = 128;   // query rows per attention tile
 
+// Record the message returned by fp_last_error() and return `st`.
+fp_status set_error(fp_status st, const char* fmt, ...);
+
 cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st);
 cudaError_t launch_search(const SearchParams& p, cudaStream_t st);
 cudaError_t launch_validate(const ValidateParams& p, cudaStream_t st);

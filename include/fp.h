@@ -142,6 +142,24 @@ FP_API fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const voi
                             float softmax_scale, void* workspace, int64_t workspace_bytes, void* out, float* lse,
                             int32_t* dev_status, void* stream);
 
+/* Largest intermediate size (bytes) fp_sparse_prefill_noalloc handles: 64 MiB. */
+#define FP_NOALLOC_MAX_BYTES (64ll << 20)
+
+/* fp_sparse_prefill for callers that cannot allocate device memory (the method on the pages has no
+ * counterpart: this is a library convenience). Serving loops that plan all device memory up front,
+ * plugin hosts that give an operator no workspace, and code that cannot afford cudaMalloc's implicit
+ * device synchronisation can call this instead: the intermediates live in a static array of
+ * FP_NOALLOC_MAX_BYTES in the library's device image, and nothing is allocated by the call.
+ * Every GPU that loads the library holds that array until the process exits. All calls on a device
+ * share it and it keeps the last call's contents (nothing needs to start at zero); calls that overlap
+ * on the GPU (other streams or threads) race on it. The first call on a device looks up the array's
+ * address with that device current: make it before any stream capture. Problems whose intermediates
+ * (fp_sparse_prefill_workspace) exceed FP_NOALLOC_MAX_BYTES return FP_ERR_INVALID_ARG.
+ * Arguments as for fp_sparse_prefill, without the workspace. */
+FP_API fp_status fp_sparse_prefill_noalloc(const fp_problem* p, const void* q, const void* k, const void* v,
+                                    float tau, float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                                    void* stream);
+
 /* Device-side check of index lists: every row's count in [1, i+1], entries ascending, in [0, i],
  * first entry 0 and last entry i. Violations OR FP_DEV_BAD_LIST into dev_status (required). */
 FP_API fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices,
