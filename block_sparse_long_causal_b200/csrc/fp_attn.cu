@@ -59,6 +59,8 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 // end marker per item).
 constexpr int kRing = 32;
 constexpr int kItemEnd = -1;
+// Largest row sum of one item that the fast path (no max pass) accepts; see the softmax loop.
+constexpr float kFastSumLimit = 65536.f;
 
 __device__ __forceinline__ uint32_t tmem_s(int k) { return 128u * k; }
 __device__ __forceinline__ uint32_t tmem_o(int k) { return 256u + 128u * k; }
@@ -473,97 +475,142 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
         if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
-        uint32_t sr[BK];
-#pragma unroll
-        for (int c = 0; c < BK; c += 32)
-          tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sr[c]));
-        tmem_wait_ld();
         // causal mask (diagonal tiles) and the list mask of this row's query block
         const int valid = ((mask >> mbit) & 1) ? (qpos - j * BK) : -1;
         const bool masked = valid < BK - 1;
-        float mx;
-        {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (masked) {
+        const uint64_t scale2 = f2_make(p.scale_log2, p.scale_log2);
+        uint32_t pk[BK / 2];
+        // Fast path, for unmasked items once the row has a reference max: no max pass. S streams
+        // from TMEM in 32-column chunks (the next chunk loads while this one is exponentiated)
+        // against the current reference max, and the item's row sum decides afterwards: a sum of
+        // at most 2^16 bounds every P below 2^16 (finite, and exact in the shared scale), so the
+        // item stands without a rescale. A larger (or non-finite) sum sends the warp through the
+        // exact path below, which reloads S (still in TMEM: P is stored only at the end).
+        bool done = false;
+        if (__all_sync(kFull, !masked && m_run != -INFINITY)) {
+          const uint64_t negm2 = f2_make(-m_run, -m_run);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+          uint32_t cb[2][32];
+          tmem_ld32(s_col, cb[0]);
 #pragma unroll
-            for (int c = 0; c < BK; ++c) {
-              const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
-              sr[c] = __float_as_uint(v);
-              m4[c & 3] = fmaxf(m4[c & 3], v);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < BK; c += 8) {
-#pragma unroll
-              for (int a = 0; a < 4; ++a)
-                m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
-            }
-          }
-          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-        }
-        const float m_new = fmaxf(m_run, mx * p.scale_log2);
-        // grow the reference max only when it rises by more than 2^8 (lazy rescale); the stale
-        // max is exact because the numerator and the denominator share it
-        const bool grow = m_new > m_run + 8.0f;
-        float alpha = 1.f;
-        if (grow) {
-          alpha = ex2_approx(m_run - m_new);
-          m_run = m_new;
-        }
-        l_run *= alpha;
-        if (n > 0 && __any_sync(kFull, grow)) {
-          // S_k(n) was committed after PV_k(n-1): O_k is complete; lanes that did not grow scale by 1
-          const uint64_t a2 = f2_make(alpha, alpha);
-#pragma unroll 1
-          for (int c = 0; c < kHeadDim; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(o_col + c, o);
+          for (int c = 0; c < BK / 32; ++c) {
             tmem_wait_ld();
+            reg_fence32(cb[c & 1]);
+            if (c + 1 < BK / 32) tmem_ld32(s_col + 32 * (c + 1), cb[(c + 1) & 1]);
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              float lo, hi;
-              f2_split(fmul2(f2_bits(o[e], o[e + 1]), a2), lo, hi);
-              o[e] = __float_as_uint(lo);
-              o[e + 1] = __float_as_uint(hi);
+              const int pr = 16 * c + e / 2;  // pair index within the item
+              const uint64_t x2 = ffma2(f2_bits(cb[c & 1][e], cb[c & 1][e + 1]), scale2, negm2);
+              uint64_t p2;
+              if ((kPolyPairs >> (pr & 7)) & 1) {
+                p2 = exp2_poly2(x2);
+              } else {
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+              }
+              acc[pr & 3] = fadd2(acc[pr & 3], p2);
+              float p0, p1;
+              f2_split(p2, p0, p1);
+              pk[pr] = pack_bf16x2(p0, p1);
             }
-            tmem_st32(o_col + c, o);
           }
+          float a0, a1, b0, b1;
+          f2_split(fadd2(acc[0], acc[1]), a0, a1);
+          f2_split(fadd2(acc[2], acc[3]), b0, b1);
+          const float isum = (a0 + a1) + (b0 + b1);
+          done = __all_sync(kFull, isum <= kFastSumLimit);
+          if (done) l_run += isum;
         }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        const uint64_t scale2 = f2_make(p.scale_log2, p.scale_log2);
-        const uint64_t negm2 = f2_make(-m_use, -m_use);
-        uint64_t sum2[2] = {0ull, 0ull};
-        uint32_t pk[BK / 2];
-        if (masked) {
-          // exact zeros for masked keys: MUFU ex2(-inf) = 0
+        if (!done) {
+          uint32_t sr[BK];
 #pragma unroll
-          for (int c = 0; c < BK; c += 2) {
-            float x0, x1;
-            f2_split(ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2), x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2_make(p0, p1));
-            pk[c / 2] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          // split exp2 between MUFU and the FMA-pipe polynomial so neither unit alone bounds it
+          for (int c = 0; c < BK; c += 32)
+            tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sr[c]));
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < BK; c += 2) {
-            const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
-            uint64_t p2;
-            if ((kPolyPairs >> ((c >> 1) & 7)) & 1) {
-              p2 = exp2_poly2(x2);
+          for (int c = 0; c < BK; c += 32) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[c]));
+          float mx;
+          {
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (masked) {
+#pragma unroll
+              for (int c = 0; c < BK; ++c) {
+                const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
+                sr[c] = __float_as_uint(v);
+                m4[c & 3] = fmaxf(m4[c & 3], v);
+              }
             } else {
-              float x0, x1;
-              f2_split(x2, x0, x1);
-              p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+#pragma unroll
+              for (int c = 0; c < BK; c += 8) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                  m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
+              }
             }
-            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
-            float p0, p1;
-            f2_split(p2, p0, p1);
-            pk[c / 2] = pack_bf16x2(p0, p1);
+            mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
           }
-        }
-        {
+          const float m_new = fmaxf(m_run, mx * p.scale_log2);
+          // grow the reference max only when it rises by more than 2^8 (lazy rescale); the stale
+          // max is exact because the numerator and the denominator share it
+          const bool grow = m_new > m_run + 8.0f;
+          float alpha = 1.f;
+          if (grow) {
+            alpha = ex2_approx(m_run - m_new);
+            m_run = m_new;
+          }
+          l_run *= alpha;
+          if (n > 0 && __any_sync(kFull, grow)) {
+            // S_k(n) was committed after PV_k(n-1): O_k is complete; lanes that did not grow scale by 1
+            const uint64_t a2 = f2_make(alpha, alpha);
+#pragma unroll 1
+            for (int c = 0; c < kHeadDim; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(o_col + c, o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float lo, hi;
+                f2_split(fmul2(f2_bits(o[e], o[e + 1]), a2), lo, hi);
+                o[e] = __float_as_uint(lo);
+                o[e + 1] = __float_as_uint(hi);
+              }
+              tmem_st32(o_col + c, o);
+            }
+          }
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          const uint64_t negm2 = f2_make(-m_use, -m_use);
+          uint64_t sum2[2] = {0ull, 0ull};
+          if (masked) {
+            // exact zeros for masked keys: MUFU ex2(-inf) = 0
+#pragma unroll
+            for (int c = 0; c < BK; c += 2) {
+              float x0, x1;
+              f2_split(ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2_make(p0, p1));
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+          } else {
+            // split exp2 between MUFU and the FMA-pipe polynomial so neither unit alone bounds it
+#pragma unroll
+            for (int c = 0; c < BK; c += 2) {
+              const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
+              uint64_t p2;
+              if ((kPolyPairs >> ((c >> 1) & 7)) & 1) {
+                p2 = exp2_poly2(x2);
+              } else {
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+              }
+              sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
+              float p0, p1;
+              f2_split(p2, p0, p1);
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+          }
           float a0, a1, b0, b1;
           f2_split(sum2[0], a0, a1);
           f2_split(sum2[1], b0, b1);
