@@ -47,8 +47,11 @@ constexpr int kRegsCtl = 104;       // WG0 (producer, MMA, idle)
 constexpr int kRegsSoftmax = 200;  // WG1, WG2
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * 168,
               "register split must equal the launch allocation");
-// exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU: 3 of 8
-constexpr unsigned kPolyPairs = 0xA4u;
+// exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU. Measured on the
+// 128K causal workload, each poly pair lengthens the softmax's dependency chains more than it
+// relieves MUFU (0 of 8: 187 M cycles per CTA, 2/8: 201 M, 3/8: 205 M, 4/8: 210 M), so every exp2
+// currently goes to MUFU; the split stays for when MUFU throughput becomes the bound.
+constexpr unsigned kPolyPairs = 0x00u;
 // Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 // Item ring: the producer merges the index lists once and publishes each kv item as
