@@ -158,6 +158,24 @@ def dist_env():
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def replica_workload(w, rank: int):
+    """The workload of one replica: same shapes, rank-distinct seeds (rank 0 keeps the originals)."""
+    return w if rank == 0 else w.with_lens(w.lens, seeds=[s + 1000 * rank for s in w.seeds])
+
+
+def reduce_over_ranks(work: list[float], times: list[float], dist=None, device="cpu"):
+    """Whole-job totals of a replica run: the work units summed over ranks and the timings maxed over
+    ranks (every rank calls this once, with lists of the same lengths, so the collectives match)."""
+    if dist is None:
+        return list(work), list(times)
+    import torch
+    w = torch.tensor(work, dtype=torch.float64, device=device)
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return w.tolist(), t.tolist()
+
+
 def run_ours(args):
     import torch
 
@@ -174,8 +192,7 @@ def run_ours(args):
 
     w = workload(args)
     tau = w.tau if args.tau is None else args.tau
-    if ws > 1:  # independent replica per rank: distinct seeds
-        w = w.with_lens(w.lens, seeds=[s + 1000 * rank for s in w.seeds])
+    w = replica_workload(w, rank)  # independent replica per rank: distinct seeds
     x = synth.make_inputs(w)
     cu = x["cu_seqlens"]
     p = fp.problem(cu, w.hq, w.hkv, w.d, w.block)
@@ -284,22 +301,20 @@ def run_ours(args):
         d2h = oh.numel() * 2
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
-    # max over ranks
+    # whole job: kept-block FLOPs summed over ranks, times maxed over ranks
     ms_step = total_ms / args.steps
-    if dist:
-        t = torch.tensor([ms_step, attn_ms, pool_ms, search_ms, e2e["ms"] if e2e else 0.0,
-                          dense_ms or 0.0], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, attn_ms, pool_ms, search_ms, e2e_max, dense_ms_max = t.tolist()
-        if e2e:
-            e2e["ms"] = e2e_max
-        if dense_ms is not None:
-            dense_ms = dense_ms_max
+    (job_flops,), (ms_step, attn_ms, pool_ms, search_ms, e2e_max, dense_ms_max) = reduce_over_ranks(
+        [eff_flops], [ms_step, attn_ms, pool_ms, search_ms, e2e["ms"] if e2e else 0.0, dense_ms or 0.0],
+        dist, device="cuda")
+    if e2e:
+        e2e["ms"] = e2e_max
+    if dense_ms is not None:
+        dense_ms = dense_ms_max
 
     pk = peaks()
     peak_tf = pk["bf16_tflops_sustained"]
     attn_tflops = eff_flops / (attn_ms * 1e-3) / 1e12
-    value = ws * eff_flops / (ms_step * 1e-3) / 1e12
+    value = job_flops / (ms_step * 1e-3) / 1e12
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -347,7 +362,7 @@ def run_ours(args):
                                "frac": round(search_bytes / (s_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                                "bytes": search_bytes}
     if e2e:
-        line["e2e"] = {"value": round(ws * eff_flops / (e2e["ms"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        line["e2e"] = {"value": round(job_flops / (e2e["ms"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                        "ms_per_step": round(e2e["ms"], 3), "h2d_bytes_per_step": e2e["h2d"],
                        "d2h_bytes_per_step": e2e["d2h"]}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
