@@ -15,9 +15,10 @@
 //                SW128 descriptor), in the pingpong order PV0(n-1) QK0(n) PV1(n-1) QK1(n).
 //        warps 2-3: idle (they only give their registers to the softmax warpgroups).
 //   WG1, WG2  softmax of slot 0 / slot 1: thread r owns query row r of its slot's tile (its TMEM
-//                lane): tcgen05.ld of S, causal mask on diagonal tiles, running max in log2 units,
-//                exp2 split between MUFU and an FMA-pipe polynomial, P packed to bf16 back into the
-//                S columns, lazy O rescale (only when the max grows by more than 2^8), final
+//                lane): tcgen05.ld of S, causal mask on diagonal tiles, running max in log2 units
+//                (no max pass on unmasked items once the row has one), exp2 on MUFU (an FMA-pipe
+//                polynomial can take a share, kPolyPairs), P packed to bf16 back into the S
+//                columns, lazy O rescale (only when the max grows by more than 2^8), final
 //                normalisation and the bf16 store of O and the LSE.
 // Registers: setmaxnreg moves WG0 down to 104 and WG1/WG2 up to 200 per thread
 // (128*104 + 256*200 = 384*168, the launch allocation of __launch_bounds__(384, 1)).
