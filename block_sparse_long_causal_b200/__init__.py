@@ -13,6 +13,9 @@ Entry points mirror the C ABI in include/fp.h:
     dense_attn(...)         -> fp_dense_attn
     sparse_prefill(...)     -> fp_sparse_prefill (all three steps, caller workspace)
     validate_lists(...)     -> fp_validate_lists
+    paged_cache(...)        -> PagedCache (fp_paged_cache_init: chunked prefill onto a paged K/V cache)
+    paged_block_pool / paged_block_search / paged_block_sparse_attn / paged_dense_attn /
+    paged_validate_lists    -> the fp_paged_* calls
 and SparsePrefill bundles the three steps with caller-side buffers.
 """
 from __future__ import annotations
@@ -32,7 +35,9 @@ FP_MAX_SEQS = 1024
 FP_NOALLOC_MAX_BYTES = 64 << 20
 EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_pool_search", "fp_block_sparse_attn",
             "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill", "fp_sparse_prefill_noalloc",
-            "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version")
+            "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version", "fp_paged_cache_init",
+            "fp_paged_block_pool", "fp_paged_block_search", "fp_paged_block_sparse_attn", "fp_paged_dense_attn",
+            "fp_paged_validate_lists")
 
 
 class FpError(RuntimeError):
@@ -48,13 +53,26 @@ class fp_problem(C.Structure):
                 ("block_size", C.c_int32)]
 
 
+class fp_paged_cache(C.Structure):
+    _fields_ = [("prefix_lens", C.c_void_p), ("block_table", C.c_void_p), ("max_pages", C.c_int32),
+                ("page_size", C.c_int32), ("num_pages", C.c_int32), ("total_kv_blocks", C.c_int32),
+                ("index_elems", C.c_int64)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libfp.so is not built ({LIB_PATH}); run python block_sparse_long_causal_b200/build.py")
     lib = C.CDLL(LIB_PATH)
     vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
     P = C.POINTER(fp_problem)
+    PC = C.POINTER(fp_paged_cache)
     sig = {
+        "fp_paged_cache_init": [PC, P, vp, vp, vp, vp, i32, i32, i32],
+        "fp_paged_block_pool": [P, PC, vp, vp, vp, vp, vp],
+        "fp_paged_block_search": [P, PC, vp, vp, f32, vp, vp, vp, vp],
+        "fp_paged_block_sparse_attn": [P, PC, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
+        "fp_paged_dense_attn": [P, PC, vp, vp, vp, f32, vp, vp, vp, vp],
+        "fp_paged_validate_lists": [P, PC, vp, vp, vp, vp],
         "fp_problem_init": [P, vp, i32, vp, i32, i32, i32, i32],
         "fp_block_pool": [P, vp, vp, vp, vp, vp],
         "fp_block_search": [P, vp, vp, f32, vp, vp, vp, vp],
@@ -188,6 +206,69 @@ def sparse_prefill_noalloc(p: Problem, q, k, v, tau: float, softmax_scale: float
 
 def selftest_exp2(x, y_poly, y_mufu, stream=None):
     _check(_lib.fp_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(), _stream(stream)))
+
+
+class PagedCache:
+    """fp_paged_cache plus the device prefix-length and block-table tensors it points to."""
+
+    def __init__(self, p: Problem, prefix_lens_host, prefix_lens_dev: torch.Tensor, block_table_dev: torch.Tensor,
+                 page_size: int, num_pages: int):
+        pre = np.ascontiguousarray(prefix_lens_host, np.int32)
+        if prefix_lens_dev.dtype != torch.int32 or block_table_dev.dtype != torch.int32:
+            raise ValueError("prefix_lens and block_table must be int32")
+        if block_table_dev.dim() != 2 or block_table_dev.shape[0] != p.num_seqs:
+            raise ValueError("block_table must be [num_seqs, max_pages]")
+        self.p = p
+        self.prefix_host = pre
+        self.prefix_dev = prefix_lens_dev
+        self.table_dev = block_table_dev.contiguous()
+        self.c = fp_paged_cache()
+        _check(_lib.fp_paged_cache_init(C.byref(self.c), p.ref, p.cu_host.ctypes.data_as(C.c_void_p),
+                                        pre.ctypes.data_as(C.c_void_p), _ptr(prefix_lens_dev), _ptr(self.table_dev),
+                                        int(self.table_dev.shape[1]), int(page_size), int(num_pages)))
+
+    def __getattr__(self, name):
+        return getattr(self.__dict__["c"], name)
+
+    @property
+    def ref(self):
+        return C.byref(self.c)
+
+
+def paged_cache(p: Problem, prefix_lens_host, block_table, page_size: int, num_pages: int, device="cuda") -> PagedCache:
+    pre = np.ascontiguousarray(prefix_lens_host, np.int32)
+    table = block_table if isinstance(block_table, torch.Tensor) else torch.from_numpy(
+        np.ascontiguousarray(block_table, np.int32))
+    return PagedCache(p, pre, torch.from_numpy(pre.copy()).to(device), table.to(device=device, dtype=torch.int32),
+                      page_size, num_pages)
+
+
+def paged_block_pool(p: Problem, c: PagedCache, q, k_cache, q_pool, k_pool, stream=None):
+    _check(_lib.fp_paged_block_pool(p.ref, c.ref, _ptr(q), _ptr(k_cache), _ptr(q_pool), _ptr(k_pool), _stream(stream)))
+
+
+def paged_block_search(p: Problem, c: PagedCache, q_pool, k_pool, tau: float, counts, indices, dev_status=None,
+                       stream=None):
+    _check(_lib.fp_paged_block_search(p.ref, c.ref, _ptr(q_pool), _ptr(k_pool), float(tau), _ptr(counts),
+                                      _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
+def paged_block_sparse_attn(p: Problem, c: PagedCache, q, k_cache, v_cache, counts, indices, softmax_scale: float, out,
+                            lse=None, dev_status=None, stream=None):
+    _check(_lib.fp_paged_block_sparse_attn(p.ref, c.ref, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(counts),
+                                           _ptr(indices), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status),
+                                           _stream(stream)))
+
+
+def paged_dense_attn(p: Problem, c: PagedCache, q, k_cache, v_cache, softmax_scale: float, out, lse=None,
+                     dev_status=None, stream=None):
+    _check(_lib.fp_paged_dense_attn(p.ref, c.ref, _ptr(q), _ptr(k_cache), _ptr(v_cache), float(softmax_scale),
+                                    _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
+def paged_validate_lists(p: Problem, c: PagedCache, counts, indices, dev_status, stream=None):
+    _check(_lib.fp_paged_validate_lists(p.ref, c.ref, _ptr(counts), _ptr(indices), _ptr(dev_status),
+                                        _stream(stream)))
 
 
 class SparsePrefill:

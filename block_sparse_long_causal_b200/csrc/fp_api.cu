@@ -40,15 +40,36 @@ fp_status check_problem(const fp_problem* p) {
   return FP_OK;
 }
 
-fp::SeqInfo seq_info(const fp_problem* p) {
+fp_status check_cache(const fp_problem* p, const fp_paged_cache* c) {
+  if (!c) return FP_OK;
+  if (!c->prefix_lens || !c->block_table)
+    return fail(FP_ERR_INVALID_ARG, "cache.prefix_lens and cache.block_table must be non-NULL (use fp_paged_cache_init)");
+  if (c->page_size <= 0 || c->page_size % p->block_size || c->max_pages < 1 || c->num_pages < 1 ||
+      c->total_kv_blocks < p->total_blocks || c->index_elems < p->index_elems)
+    return fail(FP_ERR_INVALID_ARG, "inconsistent paged cache (use fp_paged_cache_init)");
+  return FP_OK;
+}
+
+// c == NULL: a plain prefill (keys = the queries' tokens, K/V indexed by cu_seqlens)
+fp::SeqInfo seq_info(const fp_problem* p, const fp_paged_cache* c = nullptr) {
   fp::SeqInfo s;
+  memset(&s, 0, sizeof s);
   s.cu_seqlens = p->cu_seqlens;
   s.num_seqs = p->num_seqs;
   s.total_tokens = p->total_tokens;
   s.total_blocks = p->total_blocks;
   s.block = p->block_size;
+  s.total_kv_blocks = c ? c->total_kv_blocks : p->total_blocks;
+  if (c) {
+    s.prefix_lens = c->prefix_lens;
+    s.block_table = c->block_table;
+    s.max_pages = c->max_pages;
+    s.page_size = c->page_size;
+    s.num_pages = c->num_pages;
+  }
   return s;
 }
+int64_t index_elems(const fp_problem* p, const fp_paged_cache* c) { return c ? c->index_elems : p->index_elems; }
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -104,11 +125,12 @@ uint64_t wait_limit_ns() {
   return (uint64_t)(ms * 1e6) > 0 ? (uint64_t)(ms * 1e6) : 1;
 }
 
-fp_status attn_common(const fp_problem* p, const void* q, const void* k, const void* v, const int32_t* counts,
-                      const int32_t* indices, int dense, float softmax_scale, void* out, float* lse,
-                      int32_t* dev_status, void* stream) {
+fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k, const void* v,
+                      const int32_t* counts, const int32_t* indices, int dense, float softmax_scale, void* out,
+                      float* lse, int32_t* dev_status, void* stream) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
+  if ((st = check_cache(p, c)) != FP_OK) return st;
   if (!q || !k || !v || !out) return fail(FP_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
   if (!dense && (!counts || !indices)) return fail(FP_ERR_INVALID_ARG, "counts and indices must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -120,10 +142,11 @@ fp_status attn_common(const fp_problem* p, const void* q, const void* k, const v
   fp::AttnParams a;
   memset(&a, 0, sizeof a);
   const int64_t T = p->total_tokens;
+  const int64_t kv_rows = c ? (int64_t)c->num_pages * c->page_size : T;  // rows of the K/V source
   if ((st = make_tmap(&a.tm_q, q, T, (int64_t)p->num_q_heads * p->head_dim, fp::kTileM)) != FP_OK) return st;
-  if ((st = make_tmap(&a.tm_k, k, T, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
-  if ((st = make_tmap(&a.tm_v, v, T, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
-  a.seq = seq_info(p);
+  if ((st = make_tmap(&a.tm_k, k, kv_rows, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
+  if ((st = make_tmap(&a.tm_v, v, kv_rows, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
+  a.seq = seq_info(p, c);
   a.hq = p->num_q_heads;
   a.hkv = p->num_kv_heads;
   a.group = p->num_q_heads / p->num_kv_heads;
@@ -133,7 +156,7 @@ fp_status attn_common(const fp_problem* p, const void* q, const void* k, const v
   a.dense = dense;
   a.counts = counts;
   a.indices = indices;
-  a.index_elems = p->index_elems;
+  a.index_elems = index_elems(p, c);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
@@ -194,16 +217,18 @@ fp_status fp_problem_init(fp_problem* p, const int32_t* host_cu, int32_t num_seq
   return check_problem(p);
 }
 
-fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float* q_pool, float* k_pool,
-                        void* stream) {
+namespace {
+fp_status pool_impl(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k, float* q_pool,
+                    float* k_pool, void* stream) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
+  if ((st = check_cache(p, c)) != FP_OK) return st;
   if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "q, k, q_pool and k_pool must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool))
     return fail(FP_ERR_INVALID_ARG, "q, k, q_pool and k_pool must be 16-byte aligned");
   if (p->total_blocks == 0) return FP_OK;
   fp::PoolParams a;
-  a.seq = seq_info(p);
+  a.seq = seq_info(p, c);
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(k);
   a.q_pool = q_pool;
@@ -213,18 +238,24 @@ fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float
   a.q_chunks = (a.q_row + 1023) / 1024;
   a.k_chunks = (a.k_row + 1023) / 1024;
   a.dev_status = nullptr;
-  const long long items = (long long)p->total_blocks * (a.q_chunks + a.k_chunks);
+  const long long items = (long long)p->total_blocks * a.q_chunks + (long long)a.seq.total_kv_blocks * a.k_chunks;
   const long long cap = (long long)sm_count() * 16;
   const int grid = (int)(items < cap ? items : cap);
   return cuda_status(fp::launch_pool(a, grid, static_cast<cudaStream_t>(stream)), "pool launch");
 }
+}  // namespace
+
+fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k, float* q_pool, float* k_pool,
+                        void* stream) {
+  return pool_impl(p, nullptr, q, k, q_pool, k_pool, stream);
+}
 
 namespace {
-fp::SearchParams search_params(const fp_problem* p, float tau, const float* k_pool, int32_t* counts,
-                               int32_t* indices, int32_t* dev_status) {
+fp::SearchParams search_params(const fp_problem* p, const fp_paged_cache* c, float tau, const float* k_pool,
+                               int32_t* counts, int32_t* indices, int32_t* dev_status) {
   fp::SearchParams a;
   memset(&a, 0, sizeof a);
-  a.seq = seq_info(p);
+  a.seq = seq_info(p, c);
   a.k_pool = k_pool;
   a.hq = p->num_q_heads;
   a.hkv = p->num_kv_heads;
@@ -237,24 +268,30 @@ fp::SearchParams search_params(const fp_problem* p, float tau, const float* k_po
   a.log_tau = tau > 0.f ? (float)std::log((double)tau) : -INFINITY;
   a.counts = counts;
   a.indices = indices;
-  a.index_elems = p->index_elems;
+  a.index_elems = index_elems(p, c);
   a.dev_status = dev_status;
   return a;
 }
-}  // namespace
 
-fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
-                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
+fp_status search_impl(const fp_problem* p, const fp_paged_cache* c, const float* q_pool, const float* k_pool,
+                      float tau, int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
+  if ((st = check_cache(p, c)) != FP_OK) return st;
   if (!q_pool || !k_pool || !counts || !indices)
     return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, counts and indices must be non-NULL");
   if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
   if (!std::isfinite(tau)) return fail(FP_ERR_INVALID_ARG, "tau must be finite");
   if (p->total_blocks == 0) return FP_OK;
-  fp::SearchParams a = search_params(p, tau, k_pool, counts, indices, dev_status);
+  fp::SearchParams a = search_params(p, c, tau, k_pool, counts, indices, dev_status);
   a.q_pool = q_pool;
   return cuda_status(fp::launch_search(a, static_cast<cudaStream_t>(stream)), "search launch");
+}
+}  // namespace
+
+fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
+                          int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
+  return search_impl(p, nullptr, q_pool, k_pool, tau, counts, indices, dev_status, stream);
 }
 
 fp_status fp_block_pool_search(const fp_problem* p, const void* q, const void* k, float tau, float* q_pool,
@@ -268,12 +305,12 @@ fp_status fp_block_pool_search(const fp_problem* p, const void* q, const void* k
 fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,
                                const int32_t* counts, const int32_t* indices, float softmax_scale, void* out,
                                float* lse, int32_t* dev_status, void* stream) {
-  return attn_common(p, q, k, v, counts, indices, 0, softmax_scale, out, lse, dev_status, stream);
+  return attn_common(p, nullptr, q, k, v, counts, indices, 0, softmax_scale, out, lse, dev_status, stream);
 }
 
 fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
                         void* out, float* lse, int32_t* dev_status, void* stream) {
-  return attn_common(p, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
+  return attn_common(p, nullptr, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
 }
 
 namespace {
@@ -322,21 +359,107 @@ fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, c
   return fp_block_sparse_attn(p, q, k, v, counts, indices, softmax_scale, out, lse, dev_status, stream);
 }
 
-fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices, int32_t* dev_status,
-                            void* stream) {
+namespace {
+fp_status validate_impl(const fp_problem* p, const fp_paged_cache* c, const int32_t* counts, const int32_t* indices,
+                        int32_t* dev_status, void* stream) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
+  if ((st = check_cache(p, c)) != FP_OK) return st;
   if (!counts || !indices || !dev_status)
     return fail(FP_ERR_INVALID_ARG, "counts, indices and dev_status must be non-NULL");
   if (p->total_blocks == 0) return FP_OK;
   fp::ValidateParams a;
-  a.seq = seq_info(p);
+  a.seq = seq_info(p, c);
   a.hq = p->num_q_heads;
   a.counts = counts;
   a.indices = indices;
-  a.index_elems = p->index_elems;
+  a.index_elems = index_elems(p, c);
   a.dev_status = dev_status;
   return cuda_status(fp::launch_validate(a, static_cast<cudaStream_t>(stream)), "validate launch");
+}
+}  // namespace
+
+fp_status fp_validate_lists(const fp_problem* p, const int32_t* counts, const int32_t* indices, int32_t* dev_status,
+                            void* stream) {
+  return validate_impl(p, nullptr, counts, indices, dev_status, stream);
+}
+
+// ---- chunked prefill onto a paged key/value cache
+fp_status fp_paged_cache_init(fp_paged_cache* c, const fp_problem* p, const int32_t* host_cu_seqlens,
+                              const int32_t* host_prefix_lens, const int32_t* dev_prefix_lens,
+                              const int32_t* dev_block_table, int32_t max_pages, int32_t page_size,
+                              int32_t num_pages) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!c || !host_cu_seqlens || !host_prefix_lens || !dev_prefix_lens || !dev_block_table)
+    return fail(FP_ERR_INVALID_ARG, "NULL argument to fp_paged_cache_init");
+  const int B = p->block_size;
+  if (page_size <= 0 || page_size % B)
+    return fail(FP_ERR_UNSUPPORTED, "page_size=%d must be a positive multiple of block_size=%d", page_size, B);
+  if (max_pages < 1 || num_pages < 1) return fail(FP_ERR_INVALID_ARG, "max_pages and num_pages must be >= 1");
+  if ((int64_t)num_pages * page_size > (int64_t)INT32_MAX)
+    return fail(FP_ERR_INVALID_ARG, "num_pages * page_size exceeds 2^31 - 1 rows");
+  if (host_cu_seqlens[p->num_seqs] != p->total_tokens)
+    return fail(FP_ERR_INVALID_ARG, "host_cu_seqlens does not match the problem");
+  int64_t kb = 0, idx = 0;
+  for (int s = 0; s < p->num_seqs; ++s) {
+    const int64_t L = (int64_t)host_cu_seqlens[s + 1] - host_cu_seqlens[s];
+    const int64_t P = host_prefix_lens[s];
+    if (L < 0) return fail(FP_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing (sequence %d)", s);
+    if (P < 0 || P % B)
+      return fail(FP_ERR_INVALID_ARG, "prefix_lens[%d]=%lld must be a non-negative multiple of block_size=%d", s,
+                  (long long)P, B);
+    if ((P + L + page_size - 1) / page_size > max_pages)
+      return fail(FP_ERR_INVALID_ARG, "sequence %d needs %lld pages, more than max_pages=%d", s,
+                  (long long)((P + L + page_size - 1) / page_size), max_pages);
+    const int64_t nb = (L + B - 1) / B, pb = P / B;
+    kb += pb + nb;
+    idx += (int64_t)p->num_q_heads * (nb * pb + nb * (nb + 1) / 2);
+  }
+  if (kb > INT32_MAX) return fail(FP_ERR_INVALID_ARG, "too many key blocks");
+  memset(c, 0, sizeof *c);
+  c->prefix_lens = dev_prefix_lens;
+  c->block_table = dev_block_table;
+  c->max_pages = max_pages;
+  c->page_size = page_size;
+  c->num_pages = num_pages;
+  c->total_kv_blocks = (int32_t)kb;
+  c->index_elems = idx;
+  return FP_OK;
+}
+
+fp_status fp_paged_block_pool(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k_cache,
+                              float* q_pool, float* k_pool, void* stream) {
+  if (!c) return fail(FP_ERR_INVALID_ARG, "cache is NULL");
+  return pool_impl(p, c, q, k_cache, q_pool, k_pool, stream);
+}
+
+fp_status fp_paged_block_search(const fp_problem* p, const fp_paged_cache* c, const float* q_pool,
+                                const float* k_pool, float tau, int32_t* counts, int32_t* indices,
+                                int32_t* dev_status, void* stream) {
+  if (!c) return fail(FP_ERR_INVALID_ARG, "cache is NULL");
+  return search_impl(p, c, q_pool, k_pool, tau, counts, indices, dev_status, stream);
+}
+
+fp_status fp_paged_block_sparse_attn(const fp_problem* p, const fp_paged_cache* c, const void* q,
+                                     const void* k_cache, const void* v_cache, const int32_t* counts,
+                                     const int32_t* indices, float softmax_scale, void* out, float* lse,
+                                     int32_t* dev_status, void* stream) {
+  if (!c) return fail(FP_ERR_INVALID_ARG, "cache is NULL");
+  return attn_common(p, c, q, k_cache, v_cache, counts, indices, 0, softmax_scale, out, lse, dev_status, stream);
+}
+
+fp_status fp_paged_dense_attn(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k_cache,
+                              const void* v_cache, float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                              void* stream) {
+  if (!c) return fail(FP_ERR_INVALID_ARG, "cache is NULL");
+  return attn_common(p, c, q, k_cache, v_cache, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
+}
+
+fp_status fp_paged_validate_lists(const fp_problem* p, const fp_paged_cache* c, const int32_t* counts,
+                                  const int32_t* indices, int32_t* dev_status, void* stream) {
+  if (!c) return fail(FP_ERR_INVALID_ARG, "cache is NULL");
+  return validate_impl(p, c, counts, indices, dev_status, stream);
 }
 
 fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
@@ -348,6 +471,6 @@ fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t
 
 const char* fp_last_error(void) { return g_err; }
 
-int32_t fp_version(void) { return 100; }
+int32_t fp_version(void) { return 200; }
 
 }  // extern "C"

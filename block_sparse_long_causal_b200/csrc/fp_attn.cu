@@ -86,8 +86,12 @@ struct Cfg {
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag, ok
   static constexpr uint32_t kOffRing = kOffMisc + 16;               // kRing int32 item entries
   static constexpr uint32_t kOffTab = (kOffRing + 4 * kRing + 15) & ~15u;
-  static constexpr uint32_t kTabBytes = 3 * 4 * (kMaxSeqs + 1) + 8 * (kMaxSeqs + 1) + 16;
-  static constexpr uint32_t kSmem = kOffTab + kTabBytes + 1024;     // + alignment slack
+  // sequence tables (5 int arrays and one int64 array of num_seqs + 1 entries), sized per launch so
+  // that the shared memory left to L1 does not shrink for the common few-sequence case
+  static constexpr uint32_t tab_bytes(int num_seqs) { return 5 * 4 * (num_seqs + 1) + 8 * (num_seqs + 1) + 16; }
+  static constexpr uint32_t smem_bytes(int num_seqs) { return kOffTab + tab_bytes(num_seqs) + 1024; }  // + alignment
+  static constexpr uint32_t kSmemMax = smem_bytes(kMaxSeqs);
+  static_assert(kSmemMax <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BK, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHeadDim, 0, 1);
 };
@@ -97,14 +101,15 @@ struct Unit {
   int s, g;         // sequence, kv-head
   int nslot;        // 1 or 2 active Q slots
   int qt[2], h[2];  // per slot: 128-row query tile (local), q-head
-  int seq0;         // first token of the sequence
-  int len, nb, gb0; // sequence length, its blocks, global id of its block 0
+  int seq0;         // first query token of the sequence
+  int len, nb, gb0; // query tokens of the sequence, its query blocks, global id of its block 0
+  int pb;           // cached prefix blocks: query block i is key block pb + i
 };
 
 // Unit order inside a sequence: kv-head outermost, then descending query tile, then the q-head
 // pairs (G even) or q-heads (G odd) of that kv-head.
-__device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s_cb, const int* s_ct, int S,
-                                            int group) {
+__device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s_cb, const int* s_ct,
+                                            const int* s_pb, int S, int group) {
   Unit u;
   u.s = find_seq(s_ct, S, t);
   const int local = t - s_ct[u.s];
@@ -112,6 +117,7 @@ __device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s
   u.len = s_cu[u.s + 1] - u.seq0;
   u.nb = s_cb[u.s + 1] - s_cb[u.s];
   u.gb0 = s_cb[u.s];
+  u.pb = s_pb[u.s];
   const int ntile = (u.len + kTileM - 1) / kTileM;
   if ((group & 1) == 0) {
     const int pairs = group / 2;
@@ -185,9 +191,9 @@ struct KvIter {
   }
 };
 
-template <int BK>
+template <int BK, bool kCache>
 __device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, const int* s_cb,
-                                            const long long* s_ib) {
+                                            const long long* s_ib, const int* s_pb) {
   KvIter it;
   it.bad = false;
   it.dense = p.dense != 0;
@@ -198,23 +204,26 @@ __device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, 
     const int k = q >> 1, hf = q & 1;
     const int blk = u.qt[k] * per + hf;
     const bool exists = k < u.nslot && hf < per && blk < u.nb;
+    const int jd = (kCache ? u.pb : 0) + blk;  // the query block's diagonal key block
     it.i[q] = 0;
-    it.lim[q] = blk;
+    it.lim[q] = jd;
     it.l[q] = nullptr;
     it.n[q] = 0;
     if (!exists) continue;
     if (it.dense) {
-      it.n[q] = blk + 1;
+      it.n[q] = jd + 1;
     } else {
-      it.l[q] = p.indices + list_row(s_cb, s_ib, u.s, u.h[k], blk);
-      it.n[q] = min(max(__ldg(p.counts + (long long)u.h[k] * NB + u.gb0 + blk), 0), blk + 1);
+      it.l[q] = p.indices + list_row(s_cb, s_ib, s_pb, u.s, u.h[k], blk);
+      it.n[q] = min(max(__ldg(p.counts + (long long)u.h[k] * NB + u.gb0 + blk), 0), jd + 1);
     }
   }
   return it;
 }
 
 // ---------------------------------------------------------------------- the kernel -------------
-template <int BK>
+// kCache: chunked prefill onto a (paged) cache; the plain prefill is compiled separately, with no
+// prefix and direct row indexing.
+template <int BK, bool kCache>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<BK>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -236,15 +245,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_ok = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
+  const int S = p.seq.num_seqs;
   int* s_cu = reinterpret_cast<int*>(smem + C::kOffTab);
-  int* s_cb = s_cu + (kMaxSeqs + 1);
-  int* s_ct = s_cb + (kMaxSeqs + 1);
-  long long* s_ib = reinterpret_cast<long long*>(smem + C::kOffTab + 12 * (kMaxSeqs + 1) + 4);
+  int* s_cb = s_cu + (S + 1);
+  int* s_ct = s_cb + (S + 1);
+  int* s_pb = s_ct + (S + 1);
+  int* s_ckb = s_pb + (S + 1);
+  long long* s_ib = reinterpret_cast<long long*>(smem + C::kOffTab + 20 * (S + 1) + 4);
   s_ib = reinterpret_cast<long long*>(((uintptr_t)s_ib + 7) & ~(uintptr_t)7);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
-  const int S = p.seq.num_seqs;
   const bool even_g = (p.group & 1) == 0;
 
   if (threadIdx.x == 0) {
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   }
   // unit table: G even -> Hq/2 units per 128 query rows; G odd -> Hq units per 256 query rows
   const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, even_g ? kTileM : 2 * kTileM,
-                                   even_g ? p.hq / 2 : p.hq, s_ok, p.dev_status) &&
+                                   even_g ? p.hq / 2 : p.hq, s_ok, p.dev_status, s_pb, s_ckb) &&
                   (p.dense || s_ib[S] == p.index_elems);
   tc_fence_before();
   __syncthreads();
@@ -298,11 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       uint32_t xit = 0;           // item-ring entries published
       int uc = 0, q_issued = 0;   // units started / Q loads issued
       bool fail = false;
-      bool bad_list = false;
+      bool bad_list = false, bad_page = false;
       for (int k = 0;; ++k, ++uc) {
         const int t = unit_of(k);
         if (t >= num_units || fail) break;
-        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
         if (!mbar_wait(b_q_empty, (uc & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
         mbar_arrive_expect_tx(b_q_full, C::kQBytes * u.nslot);
         for (int sl = 0; sl < u.nslot; ++sl) {
@@ -311,32 +322,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           tma_load_2d(sQ + sl * C::kQBytes + C::kSlabQ, &p.tm_q, b_q_full, u.h[sl] * kHeadDim + 64, y);
         }
         ++q_issued;
-        KvIter itr = make_iter<BK>(p, u, s_cb, s_ib);
+        KvIter itr = make_iter<BK, kCache>(p, u, s_cb, s_ib, s_pb);
         int j, mask;
         while (true) {
-          const bool more = itr.next(j, mask);
+          bool more = itr.next(j, mask);
+          long long y = (long long)u.seq0 + j * BK;  // first K/V row of key block j
+          if constexpr (kCache) {  // pages hold whole blocks
+            while (more && (y = kv_row(p.seq, s_cu, u.s, j * BK)) < 0) {
+              bad_page = true;  // block table outside the cache: the block is skipped
+              more = itr.next(j, mask);
+            }
+          }
           s_item[xit % kRing] = more ? (j << 4) | mask : kItemEnd;  // publish the item (or the unit's end)
           mbar_arrive(b_item(xit));
           ++xit;
           if (!more) break;
-          const int y = u.seq0 + j * BK;
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_empty(ks), ((kit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
           mbar_arrive_expect_tx(b_k_full(ks), C::kKVBytes);
-          tma_load_2d(sK + ks * C::kKVBytes, &p.tm_k, b_k_full(ks), u.g * kHeadDim, y);
-          tma_load_2d(sK + ks * C::kKVBytes + C::kSlabKV, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, y);
+          tma_load_2d(sK + ks * C::kKVBytes, &p.tm_k, b_k_full(ks), u.g * kHeadDim, (int32_t)y);
+          tma_load_2d(sK + ks * C::kKVBytes + C::kSlabKV, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, (int32_t)y);
           ++kit;
           const int vs = vit % C::kStages;
           if (!mbar_wait(b_v_empty(vs), ((vit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
           mbar_arrive_expect_tx(b_v_full(vs), C::kKVBytes);
-          tma_load_2d(sV + vs * C::kKVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, y);
-          tma_load_2d(sV + vs * C::kKVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, y);
+          tma_load_2d(sV + vs * C::kKVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, (int32_t)y);
+          tma_load_2d(sV + vs * C::kKVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, (int32_t)y);
           ++vit;
           if (*s_abort) { fail = true; break; }
         }
         bad_list |= itr.bad;
       }
       if (bad_list) dev_flag(p.dev_status, kDevBadList);
+      if (bad_page) dev_flag(p.dev_status, kDevBadProblem);
       if (fail) {
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
@@ -393,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       for (int k = 0;; ++k, ++uc) {
         const int t = unit_of(k);
         if (t >= num_units || fail) break;
-        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+        const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
         if (!mbar_wait(b_q_full, uc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
         int e, n = 0;
@@ -464,9 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     for (int k = 0;; ++k) {
       const int t = unit_of(k);
       if (t >= num_units || fail) break;
-      const Unit u = decode_unit(t, s_cu, s_cb, s_ct, S, p.group);
+      const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
       const bool active = slot < u.nslot;     // an idle slot only consumes the unit's ring entries
       const int qpos = u.qt[slot] * kTileM + r;  // local query position of this row
+      // Rows past the sequence end (the last tile's padding) hold whatever follows in memory: they
+      // never take part in the warp's path votes, so a sequence's outputs do not depend on its
+      // neighbours in the batch (or on what lies past the end of a cache page).
+      const bool pad = qpos >= u.len;
       float m_run = -INFINITY, l_run = 0.f;
       int n = 0;
       while (true) {
@@ -480,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
         // causal mask (diagonal tiles) and the list mask of this row's query block
-        const int valid = ((mask >> mbit) & 1) ? (qpos - j * BK) : -1;
+        const int valid = ((mask >> mbit) & 1) ? (qpos - (j - (kCache ? u.pb : 0)) * BK) : -1;
         const bool masked = valid < BK - 1;
         const uint64_t scale2 = f2_make(p.scale_log2, p.scale_log2);
         uint32_t pk[BK / 2];
@@ -491,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // item stands without a rescale. A larger (or non-finite) sum sends the warp through the
         // exact path below, which reloads S (still in TMEM: P is stored only at the end).
         bool done = false;
-        if (__all_sync(kFull, !masked && m_run != -INFINITY)) {
+        if (__all_sync(kFull, pad || (!masked && m_run != -INFINITY))) {
           const uint64_t negm2 = f2_make(-m_run, -m_run);
           uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
           uint32_t cb[2][32];
@@ -523,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           f2_split(fadd2(acc[0], acc[1]), a0, a1);
           f2_split(fadd2(acc[2], acc[3]), b0, b1);
           const float isum = (a0 + a1) + (b0 + b1);
-          done = __all_sync(kFull, isum <= kFastSumLimit);
+          done = __all_sync(kFull, pad || isum <= kFastSumLimit);
           if (done) l_run += isum;
         }
         if (!done) {
@@ -683,22 +705,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int BK>
+template <int BK, bool kCache>
 static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BK>::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<BK, kCache>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<BK>::kSmemMax);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  attn_kernel<BK><<<grid, kThreads, Cfg<BK>::kSmem, st>>>(p);
+  attn_kernel<BK, kCache><<<grid, kThreads, Cfg<BK>::smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st) {
-  if (p.seq.block == 128) return launch_attn_t<128>(p, grid, st);
-  return launch_attn_t<64>(p, grid, st);
+  const bool cache = p.seq.prefix_lens != nullptr || p.seq.block_table != nullptr;
+  if (p.seq.block == 128) return cache ? launch_attn_t<128, true>(p, grid, st) : launch_attn_t<128, false>(p, grid, st);
+  return cache ? launch_attn_t<64, true>(p, grid, st) : launch_attn_t<64, false>(p, grid, st);
 }
 
 }  // namespace fp

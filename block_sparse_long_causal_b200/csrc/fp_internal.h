@@ -10,19 +10,31 @@
 namespace fp {
 
 struct SeqInfo {
-  const int32_t* cu_seqlens;  // device [S+1]
+  const int32_t* cu_seqlens;  // device [S+1], the queries (and, without a cache, the keys)
   int32_t num_seqs;
   int32_t total_tokens;
-  int32_t total_blocks;
+  int32_t total_blocks;       // query blocks
   int32_t block;              // B
+  // Chunked prefill onto a key/value cache (all zero / null for a plain prefill): sequence s has
+  // prefix_lens[s] cached tokens (a multiple of B) before its L_s queries, so its keys are the
+  // prefix_lens[s] + L_s tokens of the cache and its query block i is key block prefix/B + i.
+  const int32_t* prefix_lens; // device [S] or null
+  int32_t total_kv_blocks;    // sum_s ceil((prefix_s + L_s) / B) (== total_blocks without a cache)
+  // Paged cache (block_table null: K/V are [total_tokens, Hkv, d] indexed by cu_seqlens):
+  // key token u of sequence s is row block_table[s * max_pages + u / page_size] * page_size +
+  // u % page_size of the cache (page_size is a multiple of B, so a key block never straddles pages).
+  const int32_t* block_table; // device [S, max_pages] or null
+  int32_t max_pages;
+  int32_t page_size;
+  int32_t num_pages;          // pages in the cache (entries outside [0, num_pages) are rejected)
 };
 
 struct PoolParams {
   SeqInfo seq;
   const uint16_t* q;          // [T, Hq, d] bf16 bits
-  const uint16_t* k;          // [T, Hkv, d]
+  const uint16_t* k;          // [T, Hkv, d], or the paged cache [pages * page_size, Hkv, d]
   float* q_pool;              // [NB, Hq, d]
-  float* k_pool;              // [NB, Hkv, d]
+  float* k_pool;              // [NBK, Hkv, d] (NBK = seq.total_kv_blocks)
   int32_t q_row;              // Hq * d
   int32_t k_row;              // Hkv * d
   int32_t q_chunks, k_chunks; // 1024-element column chunks per token row
@@ -32,7 +44,7 @@ struct PoolParams {
 struct SearchParams {
   SeqInfo seq;
   const float* q_pool;        // pooled queries [NB, Hq, d]
-  const float* k_pool;
+  const float* k_pool;        // pooled keys [NBK, Hkv, d]
   int32_t hq, hkv, group;     // group = Hq / Hkv
   int32_t rows_blocks;        // query blocks per CTA tile (TI)
   int32_t num_tiles;          // grid-size hint (upper bound); the exact count is s_ct[S] on device
@@ -40,7 +52,7 @@ struct SearchParams {
   float log_tau;              // threshold on s - max (natural log units); -inf keeps all
   int32_t keep_all;           // tau <= 0
   int32_t* counts;            // [Hq, NB]
-  int32_t* indices;           // triangular
+  int32_t* indices;           // row (s, h, i) at base_s + h*(nb*pb + nb(nb+1)/2) + i*pb + i(i+1)/2
   int64_t index_elems;
   int32_t* dev_status;
 };
@@ -56,7 +68,7 @@ struct ValidateParams {
 
 struct __align__(64) AttnParams {
   CUtensorMap tm_q;           // Q as 2-D [T rows, Hq*d cols], box {64, 128}, 128B swizzle
-  CUtensorMap tm_k;           // K as 2-D [T rows, Hkv*d cols], box {64, B}
+  CUtensorMap tm_k;           // K as 2-D [T (or pages * page_size) rows, Hkv*d cols], box {64, B}
   CUtensorMap tm_v;           // V likewise
   SeqInfo seq;
   int32_t hq, hkv, group;

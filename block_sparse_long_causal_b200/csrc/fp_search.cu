@@ -45,36 +45,62 @@ __device__ __forceinline__ uint4 ld_stream_16(const uint16_t* p) {
   return v;
 }
 
+// Sequence tables in dynamic shared memory, sized for the launch's sequence count (a few bytes for
+// one sequence), so that the many small pool CTAs all stay resident.
+__host__ __device__ inline size_t pool_smem_bytes(int num_seqs) { return (size_t)(4 * (num_seqs + 1) + 1) * 4; }
+
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolParams p) {
-  __shared__ int s_cu[kMaxSeqs + 1], s_cb[kMaxSeqs + 1];
-  __shared__ int s_ok;
-  if (!build_seq_tables(p.seq, s_cu, s_cb, nullptr, nullptr, 0, 0, 0, &s_ok, p.dev_status)) return;
+  extern __shared__ int pool_tab[];
   const int S = p.seq.num_seqs, B = p.seq.block;
-  const int per_block = p.q_chunks + p.k_chunks;
-  const long long items = (long long)p.seq.total_blocks * per_block;
+  int* s_cu = pool_tab;
+  int* s_cb = s_cu + (S + 1);
+  int* s_pb = s_cb + (S + 1);
+  int* s_ckb = s_pb + (S + 1);
+  int* s_ok = s_ckb + (S + 1);
+  if (!build_seq_tables(p.seq, s_cu, s_cb, nullptr, nullptr, 0, 0, 0, s_ok, p.dev_status, s_pb, s_ckb)) return;
+  // work items: (query block, Q column chunk) first, then (key block, K column chunk); the key
+  // blocks of a sequence cover its cached prefix and its new tokens
+  const long long q_items = (long long)p.seq.total_blocks * p.q_chunks;
+  const long long items = q_items + (long long)p.seq.total_kv_blocks * p.k_chunks;
   for (long long w = blockIdx.x; w < items; w += gridDim.x) {
-    const int gb = (int)(w / per_block);
-    const int part = (int)(w % per_block);
-    const int s = find_seq(s_cb, S, gb);
-    const int i = gb - s_cb[s];
-    const int t0 = s_cu[s] + i * B;
-    const int t1 = min(t0 + B, s_cu[s + 1]);
-    const bool is_q = part < p.q_chunks;
+    const bool is_q = w < q_items;
+    const long long wl = is_q ? w : w - q_items;
+    const int chunks = is_q ? p.q_chunks : p.k_chunks;
+    const int gb = (int)(wl / chunks);
+    const int part = (int)(wl % chunks);
+    long long r0;  // first source row of the block
+    int n;         // tokens in the block
+    if (is_q) {
+      const int s = find_seq(s_cb, S, gb);
+      const int t0 = s_cu[s] + (gb - s_cb[s]) * B;
+      r0 = t0;
+      n = min(B, s_cu[s + 1] - t0);
+    } else {
+      const int s = find_seq(s_ckb, S, gb);
+      const int u0 = (gb - s_ckb[s]) * B;
+      const int klen = s_pb[s] * B + (s_cu[s + 1] - s_cu[s]);
+      n = min(B, klen - u0);
+      r0 = kv_row(p.seq, s_cu, s, u0);  // the block's n rows are contiguous (pages hold whole blocks)
+      if (r0 < 0) {
+        if (threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
+        continue;
+      }
+    }
     const int row = is_q ? p.q_row : p.k_row;
-    const int col = (is_q ? part : part - p.q_chunks) * kPoolChunk + threadIdx.x * 8;
+    const int col = part * kPoolChunk + threadIdx.x * 8;
     if (col >= row) continue;
-    const uint16_t* src = (is_q ? p.q : p.k) + (long long)t0 * row + col;
+    const uint16_t* src = (is_q ? p.q : p.k) + r0 * row + col;
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    int t = t0;
-    for (; t + 8 <= t1; t += 8) {
+    int t = 0;
+    for (; t + 8 <= n; t += 8) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = ld_stream_16(src + (long long)(t - t0 + u) * row);
+      for (int u = 0; u < 8; ++u) v[u] = ld_stream_16(src + (long long)(t + u) * row);
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc_bf16x8(a, v[u]);
     }
-    for (; t < t1; ++t) acc_bf16x8(a, ld_stream_16(src + (long long)(t - t0) * row));
-    const float inv_n = 1.0f / (float)(t1 - t0);
+    for (; t < n; ++t) acc_bf16x8(a, ld_stream_16(src + (long long)t * row));
+    const float inv_n = 1.0f / (float)n;
     float* dst = (is_q ? p.q_pool : p.k_pool) + (long long)gb * row + col;
     float4 o0 = make_float4(a[0] * inv_n, a[1] * inv_n, a[2] * inv_n, a[3] * inv_n);
     float4 o1 = make_float4(a[4] * inv_n, a[5] * inv_n, a[6] * inv_n, a[7] * inv_n);
@@ -84,7 +110,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolParams p) 
 }
 
 cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
-  pool_kernel<<<grid, kPoolThreads, 0, st>>>(p);
+  pool_kernel<<<grid, kPoolThreads, pool_smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }
 
@@ -134,7 +160,7 @@ static_assert(2 * kKChunk * kBfStride * 2 <= (int)sizeof(float) * 2 * kKChunk * 
 static_assert(kSearchRows * (kKChunk + 1) <= kKChunk * kKStride, "score tile must fit in one key buffer");
 
 __host__ __device__ inline size_t search_smem_bytes(int num_seqs) {
-  return sizeof(SearchSmem) + (size_t)(num_seqs + 1) * (3 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
+  return sizeof(SearchSmem) + (size_t)(num_seqs + 1) * (5 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
@@ -288,9 +314,11 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
   int* t_cu = reinterpret_cast<int*>(search_smem_raw + sizeof(SearchSmem));
   int* t_cb = t_cu + (S + 1);
   int* t_ct = t_cb + (S + 1);
-  long long* t_ib = reinterpret_cast<long long*>(((uintptr_t)(t_ct + (S + 1)) + 7) & ~(uintptr_t)7);
+  int* t_pb = t_ct + (S + 1);
+  int* t_ckb = t_pb + (S + 1);
+  long long* t_ib = reinterpret_cast<long long*>(((uintptr_t)(t_ckb + (S + 1)) + 7) & ~(uintptr_t)7);
   if (!build_seq_tables(p.seq, t_cu, t_cb, t_ct, t_ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
-                        p.dev_status))
+                        p.dev_status, t_pb, t_ckb))
     return;
   if (t_ib[S] != p.index_elems) {
     if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
@@ -315,8 +343,11 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
     const int g = local % p.hkv;
     const int i0 = it * TI;
     const int i_last = min(i0 + TI, nb) - 1;
-    const int gb0 = t_cb[s];
-    const int nchunks = i_last / kKChunk + 1;
+    const int gb0 = t_cb[s];   // global query block of local block 0 (pooled queries, counts)
+    const int pb = t_pb[s];    // cached prefix blocks: query block i is key block pb + i
+    const int kb0 = t_ckb[s];  // global key block of the sequence's key block 0 (pooled keys)
+    const int jmax = pb + i_last;  // last key block any row of the tile attends
+    const int nchunks = jmax / kKChunk + 1;
 
     __syncthreads();  // previous tile done with shared memory
     const float* q_src = p.q_pool;  // pooled queries of the tile (global, L2 resident)
@@ -330,12 +361,14 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
       sm.kmax_bits = 0;
     }
 
-    // emission rows: warp w emits rows 8w..8w+7
-    int row_i[8], row_h[8];
+    // emission rows: warp w emits rows 8w..8w+7; row_i is the local query block, row_j the last
+    // key block of the row (its diagonal, pb + i), -1 for padding rows
+    int row_i[8], row_j[8], row_h[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int rr = warp * 8 + r;
       row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
+      row_j[r] = row_i[r] >= 0 ? pb + row_i[r] : -1;
       row_h[r] = g * G + rr % G;
     }
     bool all_keep[8];
@@ -355,18 +388,18 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const int r = r0 + g4 + 8 * h2;
-        ri[h2] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+        ri[h2] = (r < TI * G && i0 + r / G <= i_last) ? pb + i0 + r / G : -1;
       }
       float am[2] = {-INFINITY, -INFINITY}, an[2] = {INFINITY, INFINITY};
       float* stage = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(kvw) + kStageOffBytes);
-      issue_stage_chunk(stage, p.k_pool, gb0, g, p.hkv, 0, i_last);
-      for (int j0 = 0; j0 <= i_last; j0 += kKChunk) {
+      issue_stage_chunk(stage, p.k_pool, kb0, g, p.hkv, 0, jmax);
+      for (int j0 = 0; j0 <= jmax; j0 += kKChunk) {
         cp_async_wait_all();
         __syncthreads();  // staged chunk visible; previous chunk's MMAs done with the split view
         load_split_rows(kvw, [&](int jr) -> const float* { return stage + jr * kHeadDim; }, nullptr,
                         &sm.kmax_bits);
         __syncthreads();  // split view ready; staging free
-        if (j0 + kKChunk <= i_last) issue_stage_chunk(stage, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
+        if (j0 + kKChunk <= jmax) issue_stage_chunk(stage, p.k_pool, kb0, g, p.hkv, j0 + kKChunk, jmax);
         float acc[4][4];
         chunk_scores_tc(qv, kvw, warp, lane, acc);
 #pragma unroll
@@ -419,13 +452,13 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
           sm.qT[4 * d4 + 2][r] = v.z;
           sm.qT[4 * d4 + 3][r] = v.w;
         }
-        issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, 0, i_last);
-        // scoring rows of this lane
+        issue_k_chunk(sm, 0, p.k_pool, kb0, g, p.hkv, 0, jmax);
+        // scoring rows of this lane (li: the row's last key block)
         int li[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int r = 2 * lane + e;
-          li[e] = (r < TI * G && i0 + r / G <= i_last) ? i0 + r / G : -1;
+          li[e] = (r < TI * G && i0 + r / G <= i_last) ? pb + i0 + r / G : -1;
         }
         float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
         // ---- pass 1: exact row max / min of the pooled scores
@@ -433,7 +466,7 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
           const int j0 = c * kKChunk;
           if (c + 1 < nchunks) {
             __syncthreads();  // buffer (c+1)&1 no longer read
-            issue_k_chunk(sm, (c + 1) & 1, p.k_pool, gb0, g, p.hkv, j0 + kKChunk, i_last);
+            issue_k_chunk(sm, (c + 1) & 1, p.k_pool, kb0, g, p.hkv, j0 + kKChunk, jmax);
             cp_async_wait_all_but_one();
           } else {
             cp_async_wait_all();
@@ -476,16 +509,16 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
 #pragma unroll
     for (int r = 0; r < 8; ++r)
       if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
-    const int warp_imax = max(max(max(row_i[0], row_i[1]), max(row_i[2], row_i[3])),
-                              max(max(row_i[4], row_i[5]), max(row_i[6], row_i[7])));
+    const int warp_jmax = max(max(max(row_j[0], row_j[1]), max(row_j[2], row_j[3])),
+                              max(max(row_j[4], row_j[5]), max(row_j[6], row_j[7])));
     if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       if (row_i[r] < 0 || !all_keep[r]) continue;
-      const int i = row_i[r];
-      int32_t* dst = p.indices + list_row(t_cb, t_ib, s, row_h[r], i);
-      for (int j = lane; j <= i; j += 32) dst[j] = j;
-      if (lane == 0) p.counts[(long long)row_h[r] * NB + gb0 + i] = i + 1;
+      const int i = row_i[r], jl = row_j[r];
+      int32_t* dst = p.indices + list_row(t_cb, t_ib, t_pb, s, row_h[r], i);
+      for (int j = lane; j <= jl; j += 32) dst[j] = j;
+      if (lane == 0) p.counts[(long long)row_h[r] * NB + gb0 + i] = jl + 1;
     }
     __syncthreads();
     if (!sm.need_pass2) continue;
@@ -497,12 +530,12 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       cnt[r] = 0;
-      base[r] = (row_i[r] >= 0) ? list_row(t_cb, t_ib, s, row_h[r], row_i[r]) : 0;
+      base[r] = (row_i[r] >= 0) ? list_row(t_cb, t_ib, t_pb, s, row_h[r], row_i[r]) : 0;
     }
     for (int c = 0; c < nchunks; ++c) {
       const int j0 = c * kKChunk;
       __syncthreads();
-      issue_k_chunk(sm, 0, p.k_pool, gb0, g, p.hkv, j0, i_last);
+      issue_k_chunk(sm, 0, p.k_pool, kb0, g, p.hkv, j0, jmax);
       cp_async_wait_all();
       __syncthreads();
       float acc[2][8];
@@ -512,15 +545,15 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
 #pragma unroll
         for (int b = 0; b < 8; ++b) sc[2 * lane + e][8 * warp + b] = acc[e][b] * p.inv_sqrt_d;
       __syncthreads();
-      if (!warp_needs || j0 > warp_imax) continue;
+      if (!warp_needs || j0 > warp_jmax) continue;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        if (row_i[r] < 0 || all_keep[r] || j0 > row_i[r]) continue;
+        if (row_i[r] < 0 || all_keep[r] || j0 > row_j[r]) continue;
 #pragma unroll
         for (int h2 = 0; h2 < kKChunk; h2 += 32) {
           const int j = j0 + h2 + lane;
           const float v = sc[warp * 8 + r][h2 + lane];
-          const bool keep = j <= row_i[r] && (j == 0 || j == row_i[r] || v - rmx[r] >= p.log_tau);
+          const bool keep = j <= row_j[r] && (j == 0 || j == row_j[r] || v - rmx[r] >= p.log_tau);
           const unsigned bal = __ballot_sync(0xffffffffu, keep);
           if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
           cnt[r] += __popc(bal);
@@ -555,12 +588,13 @@ cudaError_t launch_search(const SearchParams& p, cudaStream_t st) {
 }
 
 // -------------------------------------------------------------------------------- validate ----
-// One warp per list row (s, h, i): count in [1, i+1]; entries ascending, in [0, i]; first 0; last i.
+// One warp per list row (s, h, i), with jd = pb + i the row's diagonal key block: count in
+// [1, jd+1]; entries ascending, in [0, jd]; first 0; last jd.
 __global__ void __launch_bounds__(256) validate_kernel(const ValidateParams p) {
-  __shared__ int s_cu[kMaxSeqs + 1], s_cb[kMaxSeqs + 1];
+  __shared__ int s_cu[kMaxSeqs + 1], s_cb[kMaxSeqs + 1], s_pb[kMaxSeqs + 1], s_ckb[kMaxSeqs + 1];
   __shared__ long long s_ib[kMaxSeqs + 1];
   __shared__ int s_ok;
-  if (!build_seq_tables(p.seq, s_cu, s_cb, nullptr, s_ib, p.hq, 0, 0, &s_ok, p.dev_status)) return;
+  if (!build_seq_tables(p.seq, s_cu, s_cb, nullptr, s_ib, p.hq, 0, 0, &s_ok, p.dev_status, s_pb, s_ckb)) return;
   if (s_ib[p.seq.num_seqs] != p.index_elems) {
     if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
     return;
@@ -572,16 +606,17 @@ __global__ void __launch_bounds__(256) validate_kernel(const ValidateParams p) {
     const int h = (int)(w / p.seq.total_blocks), gb = (int)(w % p.seq.total_blocks);
     const int s = find_seq(s_cb, p.seq.num_seqs, gb);
     const int i = gb - s_cb[s];
+    const int jd = s_pb[s] + i;
     const int n = p.counts[(long long)h * p.seq.total_blocks + gb];
-    bool bad = (n < 1 || n > i + 1);
+    bool bad = (n < 1 || n > jd + 1);
     if (!bad) {
-      const int32_t* row = p.indices + list_row(s_cb, s_ib, s, h, i);
+      const int32_t* row = p.indices + list_row(s_cb, s_ib, s_pb, s, h, i);
       for (int e = lane; e < n; e += 32) {
         const int x = row[e];
         const int prev = e > 0 ? row[e - 1] : -1;
-        if (x < 0 || x > i || x <= prev) bad = true;
+        if (x < 0 || x > jd || x <= prev) bad = true;
         if (e == 0 && x != 0) bad = true;
-        if (e == n - 1 && x != i) bad = true;
+        if (e == n - 1 && x != jd) bad = true;
       }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) dev_flag(p.dev_status, kDevBadList);

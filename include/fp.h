@@ -142,6 +142,79 @@ FP_API fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const voi
                             float softmax_scale, void* workspace, int64_t workspace_bytes, void* out, float* lse,
                             int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Chunked prefill onto a paged key/value cache (FlashPrefill V2 abstract: paged KV cache and
+ * continuous batching in a serving engine). The pages give no interface; this one keeps the method
+ * unchanged and only moves where the keys come from:
+ *   - fp_problem describes the new query tokens of this call (the chunk): cu_seqlens over the
+ *     chunk's queries, L_s of them for sequence s, and Q is [total_tokens, Hq, d] as before.
+ *   - Sequence s already holds prefix_lens[s] tokens in the cache (a multiple of block_size), and
+ *     the caller has written the chunk's own keys and values into the cache too: the keys of s are
+ *     its prefix_lens[s] + L_s cached tokens, and the chunk's query at local position t sits at key
+ *     position prefix_lens[s] + t (causal: it attends keys 0 .. prefix_lens[s] + t).
+ *   - Blocks restart at every sequence's key position 0: the chunk's query block i is key block
+ *     pb_s + i (pb_s = prefix_lens[s] / block_size), and its list keeps key blocks 0 .. pb_s + i
+ *     (sink block 0 and its diagonal pb_s + i are always kept). The prefix is therefore attended
+ *     block-sparsely like the rest of the sequence, with pooled keys computed from the cache.
+ *   - The cache: k_cache and v_cache are device bf16 [num_pages * page_size, Hkv, d] (pages of
+ *     page_size consecutive token rows). Key token u of sequence s lives in page
+ *     block_table[s * max_pages + u / page_size] at row u % page_size. page_size must be a
+ *     multiple of block_size, so a key block never straddles pages. Block-table entries outside
+ *     [0, num_pages) make the kernels skip that key block and flag FP_DEV_BAD_PROBLEM.
+ *   - Pooled keys: float32 [total_kv_blocks, Hkv, d], key block j of sequence s at global key
+ *     block sum_{s'<s}(pb_{s'} + nb_{s'}) + j. Pooled queries, counts: as for fp_block_pool /
+ *     fp_block_search (per query block of the chunk).
+ *   - indices: row (s, h, i) starts at base_s + h * (nb_s*pb_s + nb_s*(nb_s+1)/2) + i*pb_s + i*(i+1)/2,
+ *     base_s = sum_{s'<s} Hq * (nb*pb + nb(nb+1)/2), and has room for pb_s + i + 1 entries (the
+ *     triangular layout above when every prefix is 0). fp_paged_cache.index_elems is its length.
+ * With every prefix 0 and the pages holding the sequences in order, these calls compute exactly
+ * what the plain calls compute. */
+typedef struct fp_paged_cache {
+  const int32_t* prefix_lens; /* device [num_seqs] */
+  const int32_t* block_table; /* device [num_seqs, max_pages] */
+  int32_t max_pages;          /* row length of block_table */
+  int32_t page_size;          /* token rows per page; a multiple of block_size */
+  int32_t num_pages;          /* pages in k_cache / v_cache */
+  int32_t total_kv_blocks;    /* sum_s (pb_s + nb_s) */
+  int64_t index_elems;        /* int32 entries of the index buffer */
+} fp_paged_cache;
+
+/* Fill *c for problem p (the chunk) from HOST copies of cu_seqlens and prefix_lens (read only during
+ * the call) and the device arrays the kernels read. Checks alignment of every prefix to block_size,
+ * page_size, and that max_pages covers every sequence's prefix + chunk. */
+FP_API fp_status fp_paged_cache_init(fp_paged_cache* c, const fp_problem* p, const int32_t* host_cu_seqlens,
+                                     const int32_t* host_prefix_lens, const int32_t* dev_prefix_lens,
+                                     const int32_t* dev_block_table, int32_t max_pages, int32_t page_size,
+                                     int32_t num_pages);
+
+/* Step 1 for a chunk: q_pool [total_blocks, Hq, d] from the chunk's q; k_pool [total_kv_blocks, Hkv, d]
+ * from every key block of every sequence in k_cache. */
+FP_API fp_status fp_paged_block_pool(const fp_problem* p, const fp_paged_cache* c, const void* q,
+                                     const void* k_cache, float* q_pool, float* k_pool, void* stream);
+
+/* Step 2 for a chunk: as fp_block_search, with row (s, h, i) scoring key blocks 0 .. pb_s + i. */
+FP_API fp_status fp_paged_block_search(const fp_problem* p, const fp_paged_cache* c, const float* q_pool,
+                                       const float* k_pool, float tau, int32_t* counts, int32_t* indices,
+                                       int32_t* dev_status, void* stream);
+
+/* Step 3 for a chunk: block-sparse causal attention of the chunk's queries over the listed key
+ * blocks of the cache (lists of key block ids <= pb_s + i). out / lse as for fp_block_sparse_attn
+ * (over the chunk's tokens). */
+FP_API fp_status fp_paged_block_sparse_attn(const fp_problem* p, const fp_paged_cache* c, const void* q,
+                                            const void* k_cache, const void* v_cache, const int32_t* counts,
+                                            const int32_t* indices, float softmax_scale, void* out, float* lse,
+                                            int32_t* dev_status, void* stream);
+
+/* Dense causal attention of the chunk's queries over all their keys in the cache. */
+FP_API fp_status fp_paged_dense_attn(const fp_problem* p, const fp_paged_cache* c, const void* q,
+                                     const void* k_cache, const void* v_cache, float softmax_scale, void* out,
+                                     float* lse, int32_t* dev_status, void* stream);
+
+/* fp_validate_lists for chunk lists: count in [1, pb_s+i+1], ascending entries in [0, pb_s+i],
+ * first 0, last pb_s + i. */
+FP_API fp_status fp_paged_validate_lists(const fp_problem* p, const fp_paged_cache* c, const int32_t* counts,
+                                         const int32_t* indices, int32_t* dev_status, void* stream);
+
 /* Largest intermediate size (bytes) fp_sparse_prefill_noalloc handles: 64 MiB. */
 #define FP_NOALLOC_MAX_BYTES (64ll << 20)
 

@@ -121,3 +121,64 @@ def test_sparse_prefill_workspace_and_argument_checks():
     assert fp._lib.fp_sparse_prefill(*args(C.c_void_p(4096 + 16), n.value)) == fp.FP_ERR_INVALID_ARG  # not 256-aligned
     assert fp._lib.fp_sparse_prefill(*args(ok, n.value - 1)) == fp.FP_ERR_INVALID_ARG
     assert "workspace" in _err()
+
+
+def _paged(cu=(0, 300, 500), prefixes=(256, 0), hq=4, B=128, max_pages=8, page_size=256, num_pages=16):
+    st, p = _prob(cu, hq=hq, hkv=2, B=B)
+    assert st == fp.FP_OK
+    c = fp.fp_paged_cache()
+    host_cu = np.array(cu, np.int32)
+    pre = np.array(prefixes, np.int32)
+    st = fp._lib.fp_paged_cache_init(C.byref(c), C.byref(p), host_cu.ctypes.data_as(C.c_void_p),
+                                     pre.ctypes.data_as(C.c_void_p), C.c_void_p(64), C.c_void_p(128), max_pages,
+                                     page_size, num_pages)
+    return st, p, c
+
+
+def test_paged_cache_init_sizes():
+    # sequence 0: 300 new tokens after 256 cached (pb 2, nb 3); sequence 1: 200 tokens, no prefix (nb 2)
+    st, p, c = _paged()
+    assert st == fp.FP_OK, _err()
+    assert c.total_kv_blocks == (2 + 3) + (0 + 2)
+    # trapezoidal rows: hq * (nb*pb + nb(nb+1)/2) per sequence
+    assert c.index_elems == 4 * (3 * 2 + 6) + 4 * (0 + 3)
+    assert c.page_size == 256 and c.max_pages == 8 and c.num_pages == 16
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(prefixes=(200, 0)), fp.FP_ERR_INVALID_ARG),       # prefix not a multiple of B
+    (dict(prefixes=(-128, 0)), fp.FP_ERR_INVALID_ARG),
+    (dict(page_size=192), fp.FP_ERR_UNSUPPORTED),           # page not a multiple of B = 128
+    (dict(page_size=0), fp.FP_ERR_UNSUPPORTED),
+    (dict(max_pages=2), fp.FP_ERR_INVALID_ARG),             # sequence 0 needs ceil(556 / 256) = 3 pages
+    (dict(num_pages=0), fp.FP_ERR_INVALID_ARG),
+    (dict(num_pages=1 << 24, page_size=256), fp.FP_ERR_INVALID_ARG),  # rows past 2^31 - 1
+])
+def test_paged_cache_init_rejects(kw, status):
+    st, _, _ = _paged(**kw)
+    assert st == status, _err()
+
+
+def test_paged_calls_reject_a_null_cache_before_launch():
+    st, p = _prob()
+    ok = C.c_void_p(4096)
+    assert fp._lib.fp_paged_block_pool(C.byref(p), None, ok, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_paged_block_search(C.byref(p), None, ok, ok, C.c_float(0.1), ok, ok, None,
+                                         None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_paged_block_sparse_attn(C.byref(p), None, ok, ok, ok, ok, ok, C.c_float(0.0), ok, None, None,
+                                              None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_paged_dense_attn(C.byref(p), None, ok, ok, ok, C.c_float(0.0), ok, None, None,
+                                       None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_paged_validate_lists(C.byref(p), None, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
+    assert "cache" in _err()
+
+
+def test_paged_calls_check_the_cache_and_arguments():
+    st, p, c = _paged()
+    assert st == fp.FP_OK
+    ok = C.c_void_p(4096)
+    # NULL q: rejected on the host
+    assert fp._lib.fp_paged_block_pool(C.byref(p), C.byref(c), None, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
+    # a hand-edited cache inconsistent with the problem
+    c.page_size = 100
+    assert fp._lib.fp_paged_block_pool(C.byref(p), C.byref(c), ok, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
