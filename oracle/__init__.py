@@ -57,6 +57,9 @@ def lib():
             L.orc_search.restype = C.c_int
             L.orc_search.argtypes = [f64p, f64p, i32p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                      C.c_double, C.c_double, i32p, i32p, u8p]
+            L.orc_search_topp.restype = C.c_int
+            L.orc_search_topp.argtypes = [f64p, f64p, i32p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                          C.c_double, C.c_double, i32p, i32p, u8p]
             L.orc_attn_rows.restype = C.c_int
             L.orc_attn_rows.argtypes = [u16p, u16p, u16p, i32p, C.c_int, C.c_int, C.c_int, C.c_int,
                                         C.c_int, C.c_double, i32p, i32p, C.c_int64, i64p, i32p, f64p, f64p]
@@ -125,6 +128,30 @@ def search(qbar, kbar, cu, B: int, tau: float, want_band: bool = True):
                           _p(band, C.c_uint8))
     if rc:
         raise ValueError("bad search arguments")
+    return counts, indices, band
+
+
+def search_topp(qbar, kbar, cu, B: int, gamma: float, want_band: bool = True):
+    """Cumulative top-p block selection on the pooled softmax (the comparison selector).
+
+    Block j of row (h, i) is kept iff the probability mass of the strictly more probable blocks is
+    below gamma (blocks tied at the cut kept together), plus the sink and the diagonal.
+    Returns (counts, indices, band) in the layout of search().
+    """
+    qbar = np.ascontiguousarray(qbar, np.float64)
+    kbar = np.ascontiguousarray(kbar, np.float64)
+    cu = np.ascontiguousarray(cu, np.int32)
+    hq, hkv, d = qbar.shape[1], kbar.shape[1], qbar.shape[2]
+    nb = total_blocks(cu, B)
+    n = index_elems(cu, B, hq)
+    counts = np.zeros((hq, nb), np.int32)
+    indices = np.full(n, -1, np.int32)
+    band = np.zeros(n, np.uint8) if want_band else None
+    rc = lib().orc_search_topp(_p(qbar, C.c_double), _p(kbar, C.c_double), _p(cu, C.c_int32), len(cu) - 1, B,
+                               hq, hkv, d, float(gamma), TIE_BAND_REL, _p(counts, C.c_int32),
+                               _p(indices, C.c_int32), _p(band, C.c_uint8))
+    if rc:
+        raise ValueError("bad search_topp arguments")
     return counts, indices, band
 
 

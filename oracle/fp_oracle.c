@@ -147,6 +147,82 @@ int orc_pooled_row(const double* qbar, const double* kbar, const int32_t* cu, in
     return 0;
 }
 
+/* ------------------------------------------------------ top-p search (comparison) ------------ */
+/* The cumulative-probability selector that FlashPrefill sets its threshold against (FlashPrefill
+ * skill summary page, "The Problem": Top-k / Top-p need score computation, sorting and cumulative
+ * sums; FlexPrefill abstract, "Cumulative-Attention Based Index Selection": the selected indexes'
+ * attention scores must sum to a preset threshold). On the same pooled scores and causal softmax
+ * p_ij as orc_search: rank the blocks by p (largest first) and keep the smallest leading set whose
+ * probability sum reaches gamma. Written without an order among equal p values: with
+ *     D_j = sum of p_l over the blocks l with p_l > p_j   (the mass ranked strictly before j),
+ * block j is kept iff D_j < gamma, so blocks tied at the cut are kept together. The sink block 0
+ * and the diagonal block i are kept as in orc_search. gamma <= 0 keeps only those two; gamma >= 1
+ * keeps every causal block. band (optional): 1 where the decision is within reach of rounding:
+ * |D_j - gamma| <= band_rel * max(gamma, 1e-300), or a block with p within 1e-5 (relative) of p_j
+ * could change D_j across gamma. */
+static int cmp_desc(const void* a, const void* b) {
+    double x = *(const double*)a, y = *(const double*)b;
+    return (x < y) - (x > y);
+}
+
+int orc_search_topp(const double* qbar, const double* kbar, const int32_t* cu, int S, int B, int Hq,
+                    int Hkv, int d, double gamma, double band_rel, int32_t* counts, int32_t* indices,
+                    uint8_t* band) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return -1;
+    int64_t NB = orc_total_blocks(cu, S, B);
+    int64_t gb0 = 0, base = 0;
+    for (int s = 0; s < S; ++s) {
+        int64_t nb = blocks_of(cu[s + 1] - cu[s], B);
+        int64_t tri = nb * (nb + 1) / 2;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+        for (int h = 0; h < Hq; ++h) {
+            for (int64_t i = 0; i < nb; ++i) {
+                int64_t n = i + 1;
+                double* score = (double*)malloc(sizeof(double) * (size_t)(5 * n));
+                double* p = score + n;
+                double* ratio = p + n;
+                double* sorted = ratio + n;
+                double* dmass = sorted + n;
+                pooled_row(qbar, kbar, gb0, Hq, Hkv, d, h, i, score, p, ratio);
+                /* D_j: mass of the strictly larger probabilities (sort, then running sums) */
+                memcpy(sorted, p, sizeof(double) * (size_t)n);
+                qsort(sorted, (size_t)n, sizeof(double), cmp_desc);
+                for (int64_t j = 0; j < n; ++j) {
+                    /* position of the first sorted entry <= p_j: everything before it is > p_j */
+                    int64_t lo = 0, hi = n;
+                    while (lo < hi) {
+                        int64_t mid = (lo + hi) / 2;
+                        if (sorted[mid] > p[j]) lo = mid + 1; else hi = mid;
+                    }
+                    double acc = 0.0;
+                    for (int64_t r = 0; r < lo; ++r) acc += sorted[r];
+                    dmass[j] = acc;
+                }
+                int64_t row = base + (int64_t)h * tri + i * (i + 1) / 2;
+                int32_t cnt = 0;
+                for (int64_t j = 0; j <= i; ++j) {
+                    int keep = gamma >= 1.0 || dmass[j] < gamma || j == 0 || j == i;
+                    if (band) {
+                        int amb = fabs(dmass[j] - gamma) <= band_rel * (gamma > 1e-300 ? gamma : 1e-300);
+                        for (int64_t l = 0; l <= i && !amb; ++l) {
+                            if (l == j) continue;
+                            double big = p[l] > p[j] ? p[l] : p[j];
+                            if (fabs(p[l] - p[j]) <= 1e-5 * big && fabs(dmass[j] - gamma) <= p[l] + p[j]) amb = 1;
+                        }
+                        band[row + j] = (uint8_t)(gamma > 0.0 && gamma < 1.0 && amb);
+                    }
+                    if (keep) indices[row + cnt++] = (int32_t)j;
+                }
+                counts[(int64_t)h * NB + gb0 + i] = cnt;
+                free(score);
+            }
+        }
+        gb0 += nb;
+        base += (int64_t)Hq * tri;
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------- search ------------------------ */
 /* Threshold + emission. counts: [Hq, NB]; indices: triangular layout above; band (optional, same
  * layout as indices, one byte per causal (row, j)): 1 where |ratio - tau| <= band_rel * tau,
