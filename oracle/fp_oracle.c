@@ -178,37 +178,36 @@ int orc_search_topp(const double* qbar, const double* kbar, const int32_t* cu, i
         for (int h = 0; h < Hq; ++h) {
             for (int64_t i = 0; i < nb; ++i) {
                 int64_t n = i + 1;
-                double* score = (double*)malloc(sizeof(double) * (size_t)(5 * n));
+                double* score = (double*)malloc(sizeof(double) * (size_t)(6 * n + 1));
                 double* p = score + n;
                 double* ratio = p + n;
                 double* sorted = ratio + n;
                 double* dmass = sorted + n;
+                double* prefix = dmass + n; /* n + 1 entries: prefix[r] = sorted[0] + ... + sorted[r-1] */
                 pooled_row(qbar, kbar, gb0, Hq, Hkv, d, h, i, score, p, ratio);
-                /* D_j: mass of the strictly larger probabilities (sort, then running sums) */
                 memcpy(sorted, p, sizeof(double) * (size_t)n);
                 qsort(sorted, (size_t)n, sizeof(double), cmp_desc);
-                for (int64_t j = 0; j < n; ++j) {
-                    /* position of the first sorted entry <= p_j: everything before it is > p_j */
+                prefix[0] = 0.0;
+                for (int64_t r = 0; r < n; ++r) prefix[r + 1] = prefix[r] + sorted[r];
+                int64_t row = base + (int64_t)h * tri + i * (i + 1) / 2;
+                int32_t cnt = 0;
+                for (int64_t j = 0; j <= i; ++j) {
+                    /* lo = number of sorted entries strictly greater than p_j; hi = those >= p_j */
                     int64_t lo = 0, hi = n;
                     while (lo < hi) {
                         int64_t mid = (lo + hi) / 2;
                         if (sorted[mid] > p[j]) lo = mid + 1; else hi = mid;
                     }
-                    double acc = 0.0;
-                    for (int64_t r = 0; r < lo; ++r) acc += sorted[r];
-                    dmass[j] = acc;
-                }
-                int64_t row = base + (int64_t)h * tri + i * (i + 1) / 2;
-                int32_t cnt = 0;
-                for (int64_t j = 0; j <= i; ++j) {
+                    int64_t eq_end = lo;
+                    while (eq_end < n && sorted[eq_end] == p[j]) ++eq_end;
+                    dmass[j] = prefix[lo]; /* D_j: mass ranked strictly before j */
                     int keep = gamma >= 1.0 || dmass[j] < gamma || j == 0 || j == i;
                     if (band) {
                         int amb = fabs(dmass[j] - gamma) <= band_rel * (gamma > 1e-300 ? gamma : 1e-300);
-                        for (int64_t l = 0; l <= i && !amb; ++l) {
-                            if (l == j) continue;
-                            double big = p[l] > p[j] ? p[l] : p[j];
-                            if (fabs(p[l] - p[j]) <= 1e-5 * big && fabs(dmass[j] - gamma) <= p[l] + p[j]) amb = 1;
-                        }
+                        /* a value within 1e-5 (relative) of p_j on either side, or an exact tie */
+                        int near = (eq_end - lo) > 1 || (lo > 0 && sorted[lo - 1] - p[j] <= 1e-5 * sorted[lo - 1]) ||
+                                   (eq_end < n && p[j] - sorted[eq_end] <= 1e-5 * p[j]);
+                        if (near && fabs(dmass[j] - gamma) <= 2.00002 * p[j] + 1e-300) amb = 1;
                         band[row + j] = (uint8_t)(gamma > 0.0 && gamma < 1.0 && amb);
                     }
                     if (keep) indices[row + cnt++] = (int32_t)j;
