@@ -176,6 +176,54 @@ def reduce_over_ranks(work: list[float], times: list[float], dist=None, device="
     return w.tolist(), t.tolist()
 
 
+def supplementary(fp, p, sp, x, q, k, v, tau, stream, w, reps=3):
+    """Outside the timed step: (1) the cumulative top-p selector (the selection FlashPrefill's max
+    threshold replaces) against the threshold search alone, on the same pooled tensors; (2) FP8
+    attention (e4m3 Q / K with per-tensor scales, bf16 V) on the step's own lists."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    out = {}
+    counts2 = torch.zeros_like(sp.counts)
+    idx2 = torch.zeros_like(sp.indices)
+    scores = torch.empty(max(p.index_elems, 1), dtype=torch.float32, device="cuda")
+    gamma = 0.95
+    out["threshold_search_ms"] = round(timed(lambda: fp.block_search(p, sp.q_pool, sp.k_pool, tau, counts2, idx2,
+                                                                        sp.dev_status, stream)), 4)
+    out["topp_search_ms"] = round(timed(lambda: fp.block_search_topp(p, sp.q_pool, sp.k_pool, gamma, scores, counts2,
+                                                                        idx2, sp.dev_status, stream)), 4)
+    eff, dense = kept_flops(counts2[:, : p.total_blocks].cpu().numpy(), x["cu_seqlens"], w.block, w.d)
+    out["topp_gamma"] = gamma
+    out["topp_density"] = round(eff / dense, 6)
+    out["topp_scores_bytes"] = int(4 * p.index_elems)
+    del scores, counts2, idx2
+    # FP8: per-tensor scales from the absolute maxima, e4m3 codes quantised on the host
+    q32, k32 = synth.bf16_bits_to_f32(x["q"]), synth.bf16_bits_to_f32(x["k"])
+    qs, ks = float(np.abs(q32).max()) / 448.0, float(np.abs(k32).max()) / 448.0
+    qc = torch.from_numpy(synth.to_e4m3_bits(q32 / qs)).cuda()
+    kc = torch.from_numpy(synth.to_e4m3_bits(k32 / ks)).cuda()
+    del q32, k32
+    o8 = torch.empty_like(sp.out)
+    ms8 = timed(lambda: fp.block_sparse_attn_fp8(p, qc, kc, v, qs, ks, sp.counts, sp.indices, 0.0, o8, None,
+                                                 sp.dev_status, stream))
+    eff1, _ = kept_flops(sp.counts[:, : p.total_blocks].cpu().numpy(), x["cu_seqlens"], w.block, w.d)
+    out["fp8_attn_ms"] = round(ms8, 3)
+    out["fp8_attn_tflops"] = round(eff1 / (ms8 * 1e-3) / 1e12, 2)
+    out["fp8_note"] = "e4m3 Q K^T (kind::f8f6f4), bf16 P V; effective FLOPs of the kept blocks"
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -236,6 +284,8 @@ def run_ours(args):
         d1.record(stream)
         torch.cuda.synchronize()
         dense_ms = d0.elapsed_time(d1) / nd
+
+    supp = None if args.no_supplementary else supplementary(fp, p, sp, x, q, k, v, tau, stream, w)
 
     uuid = None
     try:
@@ -347,6 +397,7 @@ def run_ours(args):
                      "traffic": measured_traffic(f"attn_kernel<{w.block}>", w.name)},
         "search_roofline": None,
         "gpu_launches": 3 * args.steps,
+        "supplementary": supp,
         "dev_status": status,
         "clocks": clk,
     }
@@ -471,6 +522,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-supplementary", action="store_true",
+                    help="skip the top-p comparison and FP8 timings reported beside the step")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

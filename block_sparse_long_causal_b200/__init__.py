@@ -8,8 +8,10 @@ Entry points mirror the C ABI in include/fp.h:
     problem(...)            -> Problem (fp_problem_init)
     block_pool(...)         -> fp_block_pool
     block_search(...)       -> fp_block_search
+    block_search_topp(...)  -> fp_block_search_topp (the cumulative top-p comparison selector)
     block_pool_search(...)  -> fp_block_pool_search (steps 1 + 2 fused)
     block_sparse_attn(...)  -> fp_block_sparse_attn
+    block_sparse_attn_fp8 / dense_attn_fp8 -> e4m3 Q / K attention (fp_*_fp8)
     dense_attn(...)         -> fp_dense_attn
     sparse_prefill(...)     -> fp_sparse_prefill (all three steps, caller workspace)
     validate_lists(...)     -> fp_validate_lists
@@ -37,7 +39,7 @@ EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_poo
             "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill", "fp_sparse_prefill_noalloc",
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version", "fp_paged_cache_init",
             "fp_paged_block_pool", "fp_paged_block_search", "fp_paged_block_sparse_attn", "fp_paged_dense_attn",
-            "fp_paged_validate_lists")
+            "fp_paged_validate_lists", "fp_block_search_topp", "fp_block_sparse_attn_fp8", "fp_dense_attn_fp8")
 
 
 class FpError(RuntimeError):
@@ -68,6 +70,9 @@ def _load():
     PC = C.POINTER(fp_paged_cache)
     sig = {
         "fp_paged_cache_init": [PC, P, vp, vp, vp, vp, i32, i32, i32],
+        "fp_block_search_topp": [P, vp, vp, f32, vp, vp, vp, vp, vp],
+        "fp_block_sparse_attn_fp8": [P, vp, vp, vp, f32, f32, vp, vp, f32, vp, vp, vp, vp],
+        "fp_dense_attn_fp8": [P, vp, vp, vp, f32, f32, f32, vp, vp, vp, vp],
         "fp_paged_block_pool": [P, PC, vp, vp, vp, vp, vp],
         "fp_paged_block_search": [P, PC, vp, vp, f32, vp, vp, vp, vp],
         "fp_paged_block_sparse_attn": [P, PC, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
@@ -164,6 +169,13 @@ def block_search(p: Problem, q_pool, k_pool, tau: float, counts, indices, dev_st
                                 _ptr(dev_status), _stream(stream)))
 
 
+def block_search_topp(p: Problem, q_pool, k_pool, gamma: float, scores, counts, indices, dev_status=None,
+                      stream=None):
+    """Cumulative top-p block selection (the comparison selector); scores: float32 [index_elems] scratch."""
+    _check(_lib.fp_block_search_topp(p.ref, _ptr(q_pool), _ptr(k_pool), float(gamma), _ptr(scores), _ptr(counts),
+                                     _ptr(indices), _ptr(dev_status), _stream(stream)))
+
+
 def block_pool_search(p: Problem, q, k, tau: float, q_pool, k_pool, counts, indices, dev_status=None, stream=None):
     _check(_lib.fp_block_pool_search(p.ref, _ptr(q), _ptr(k), float(tau), _ptr(q_pool), _ptr(k_pool), _ptr(counts),
                                      _ptr(indices), _ptr(dev_status), _stream(stream)))
@@ -173,6 +185,20 @@ def block_sparse_attn(p: Problem, q, k, v, counts, indices, softmax_scale: float
                       stream=None):
     _check(_lib.fp_block_sparse_attn(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(counts), _ptr(indices),
                                      float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
+def block_sparse_attn_fp8(p: Problem, q_e4m3, k_e4m3, v, q_scale: float, k_scale: float, counts, indices,
+                          softmax_scale: float, out, lse=None, dev_status=None, stream=None):
+    """FP8 attention: e4m3 Q / K codes (uint8 tensors) with per-tensor scales, bf16 V."""
+    _check(_lib.fp_block_sparse_attn_fp8(p.ref, _ptr(q_e4m3), _ptr(k_e4m3), _ptr(v), float(q_scale), float(k_scale),
+                                         _ptr(counts), _ptr(indices), float(softmax_scale), _ptr(out), _ptr(lse),
+                                         _ptr(dev_status), _stream(stream)))
+
+
+def dense_attn_fp8(p: Problem, q_e4m3, k_e4m3, v, q_scale: float, k_scale: float, softmax_scale: float, out, lse=None,
+                   dev_status=None, stream=None):
+    _check(_lib.fp_dense_attn_fp8(p.ref, _ptr(q_e4m3), _ptr(k_e4m3), _ptr(v), float(q_scale), float(k_scale),
+                                  float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
 
 
 def dense_attn(p: Problem, q, k, v, softmax_scale: float, out, lse=None, dev_status=None, stream=None):

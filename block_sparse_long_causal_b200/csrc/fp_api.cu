@@ -96,15 +96,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [rows, cols] row-major, box {64 cols, box_rows}, 128-byte swizzle, zero fill out of range.
-fp_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+// [rows, cols] row-major, 128-byte swizzle, zero fill out of range. bf16: box {64 cols, box_rows};
+// one-byte elements (e4m3 carried as uint8): box {128 cols, box_rows}. Either way a box row is
+// one 128-byte swizzle atom.
+fp_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, bool byte_elems = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int el = byte_elems ? 1 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * el};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / el), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, byte_elems ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -125,9 +129,11 @@ uint64_t wait_limit_ns() {
   return (uint64_t)(ms * 1e6) > 0 ? (uint64_t)(ms * 1e6) : 1;
 }
 
+// fp8: q and k hold e4m3 codes (one byte per element) and the logits are
+// softmax_scale * (qk_scale * q . k), qk_scale = q_scale * k_scale.
 fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k, const void* v,
                       const int32_t* counts, const int32_t* indices, int dense, float softmax_scale, void* out,
-                      float* lse, int32_t* dev_status, void* stream) {
+                      float* lse, int32_t* dev_status, void* stream, bool fp8 = false, float qk_scale = 1.f) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
   if ((st = check_cache(p, c)) != FP_OK) return st;
@@ -143,8 +149,9 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   memset(&a, 0, sizeof a);
   const int64_t T = p->total_tokens;
   const int64_t kv_rows = c ? (int64_t)c->num_pages * c->page_size : T;  // rows of the K/V source
-  if ((st = make_tmap(&a.tm_q, q, T, (int64_t)p->num_q_heads * p->head_dim, fp::kTileM)) != FP_OK) return st;
-  if ((st = make_tmap(&a.tm_k, k, kv_rows, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
+  if ((st = make_tmap(&a.tm_q, q, T, (int64_t)p->num_q_heads * p->head_dim, fp::kTileM, fp8)) != FP_OK) return st;
+  if ((st = make_tmap(&a.tm_k, k, kv_rows, (int64_t)p->num_kv_heads * p->head_dim, p->block_size, fp8)) != FP_OK)
+    return st;
   if ((st = make_tmap(&a.tm_v, v, kv_rows, (int64_t)p->num_kv_heads * p->head_dim, p->block_size)) != FP_OK) return st;
   a.seq = seq_info(p, c);
   a.hq = p->num_q_heads;
@@ -157,7 +164,8 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   a.counts = counts;
   a.indices = indices;
   a.index_elems = index_elems(p, c);
-  a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale_log2 = scale * qk_scale * 1.4426950408889634f;
+  a.fp8 = fp8 ? 1 : 0;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.dev_status = dev_status;
@@ -294,6 +302,21 @@ fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float*
   return search_impl(p, nullptr, q_pool, k_pool, tau, counts, indices, dev_status, stream);
 }
 
+fp_status fp_block_search_topp(const fp_problem* p, const float* q_pool, const float* k_pool, float gamma,
+                               float* scores, int32_t* counts, int32_t* indices, int32_t* dev_status,
+                               void* stream) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if (!q_pool || !k_pool || !scores || !counts || !indices)
+    return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, scores, counts and indices must be non-NULL");
+  if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
+  if (!std::isfinite(gamma)) return fail(FP_ERR_INVALID_ARG, "gamma must be finite");
+  if (p->total_blocks == 0) return FP_OK;
+  fp::SearchParams a = search_params(p, nullptr, gamma, k_pool, counts, indices, dev_status);
+  a.q_pool = q_pool;
+  return cuda_status(fp::launch_topp(a, gamma, scores, static_cast<cudaStream_t>(stream)), "top-p search launch");
+}
+
 fp_status fp_block_pool_search(const fp_problem* p, const void* q, const void* k, float tau, float* q_pool,
                                float* k_pool, int32_t* counts, int32_t* indices, int32_t* dev_status,
                                void* stream) {
@@ -311,6 +334,35 @@ fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k
 fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
                         void* out, float* lse, int32_t* dev_status, void* stream) {
   return attn_common(p, nullptr, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream);
+}
+
+namespace {
+fp_status check_fp8_scales(float q_scale, float k_scale, float* qk) {
+  if (!std::isfinite(q_scale) || !std::isfinite(k_scale) || !(q_scale > 0.f) || !(k_scale > 0.f))
+    return fail(FP_ERR_INVALID_ARG, "q_scale and k_scale must be finite and positive");
+  *qk = q_scale * k_scale;
+  if (!std::isfinite(*qk) || !(*qk > 0.f)) return fail(FP_ERR_INVALID_ARG, "q_scale * k_scale out of range");
+  return FP_OK;
+}
+}  // namespace
+
+fp_status fp_block_sparse_attn_fp8(const fp_problem* p, const void* q, const void* k, const void* v, float q_scale,
+                                   float k_scale, const int32_t* counts, const int32_t* indices, float softmax_scale,
+                                   void* out, float* lse, int32_t* dev_status, void* stream) {
+  float qk = 1.f;
+  fp_status st = check_fp8_scales(q_scale, k_scale, &qk);
+  if (st != FP_OK) return st;
+  return attn_common(p, nullptr, q, k, v, counts, indices, 0, softmax_scale, out, lse, dev_status, stream, true, qk);
+}
+
+fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q, const void* k, const void* v, float q_scale,
+                            float k_scale, float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                            void* stream) {
+  float qk = 1.f;
+  fp_status st = check_fp8_scales(q_scale, k_scale, &qk);
+  if (st != FP_OK) return st;
+  return attn_common(p, nullptr, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream, true,
+                     qk);
 }
 
 namespace {

@@ -69,17 +69,22 @@ constexpr float kFastSumLimit = 65536.f;
 __device__ __forceinline__ uint32_t tmem_s(int k) { return 128u * k; }
 __device__ __forceinline__ uint32_t tmem_o(int k) { return 256u + 128u * k; }
 
-template <int BK>
+// kFp8: Q and K are e4m3 (1 byte per element: a 128-element head row is one 128-byte swizzle
+// atom wide, so their tiles are a single slab); V and P stay bf16.
+template <int BK, bool kFp8 = false>
 struct Cfg {
   static constexpr int kStages = BK == 128 ? 2 : 4;                // K ring and V ring slots
-  static constexpr uint32_t kQBytes = kTileM * kHeadDim * 2;        // 32 KB per slot
-  static constexpr uint32_t kKVBytes = BK * kHeadDim * 2;           // one K or V tile
-  static constexpr uint32_t kSlabQ = kTileM * 128;                  // 64 cols x 2 B x rows
-  static constexpr uint32_t kSlabKV = BK * 128;
+  static constexpr uint32_t kQKEl = kFp8 ? 1 : 2;                   // bytes per Q / K element
+  static constexpr uint32_t kQBytes = kTileM * kHeadDim * kQKEl;    // one Q slot
+  static constexpr uint32_t kKBytes = BK * kHeadDim * kQKEl;        // one K tile
+  static constexpr uint32_t kVBytes = BK * kHeadDim * 2;            // one V tile
+  static constexpr uint32_t kSlabQ = kTileM * 128;                  // 128-byte rows x rows
+  static constexpr uint32_t kSlabK = BK * 128;
+  static constexpr uint32_t kSlabKV = BK * 128;                     // V slab (64 bf16 columns)
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = 2 * kQBytes;
-  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
-  static constexpr uint32_t kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKBytes;
+  static constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
   // barriers: q_full, q_empty, k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2],
   // o_final[2], drain, never (the test hook's barrier that nothing arrives on), item[kRing]
   static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2 + kRing;
@@ -92,7 +97,7 @@ struct Cfg {
   static constexpr uint32_t smem_bytes(int num_seqs) { return kOffTab + tab_bytes(num_seqs) + 1024; }  // + alignment
   static constexpr uint32_t kSmemMax = smem_bytes(kMaxSeqs);
   static_assert(kSmemMax <= 227 * 1024, "shared memory per CTA");
-  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, BK, 0, 0);
+  static constexpr uint32_t kIdescQK = kFp8 ? idesc_e4m3_f32(128, BK) : idesc_bf16_f32(128, BK, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHeadDim, 0, 1);
 };
 
@@ -222,10 +227,10 @@ __device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, 
 
 // ---------------------------------------------------------------------- the kernel -------------
 // kCache: chunked prefill onto a (paged) cache; the plain prefill is compiled separately, with no
-// prefix and direct row indexing.
-template <int BK, bool kCache>
+// prefix and direct row indexing. kFp8: e4m3 Q and K (QK^T on kind::f8f6f4), bf16 V.
+template <int BK, bool kCache, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<BK>;
+  using C = Cfg<BK, kFp8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -319,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         for (int sl = 0; sl < u.nslot; ++sl) {
           const int y = u.seq0 + u.qt[sl] * kTileM;
           tma_load_2d(sQ + sl * C::kQBytes, &p.tm_q, b_q_full, u.h[sl] * kHeadDim, y);
-          tma_load_2d(sQ + sl * C::kQBytes + C::kSlabQ, &p.tm_q, b_q_full, u.h[sl] * kHeadDim + 64, y);
+          if constexpr (!kFp8)  // bf16: the second 64 columns are a second slab
+            tma_load_2d(sQ + sl * C::kQBytes + C::kSlabQ, &p.tm_q, b_q_full, u.h[sl] * kHeadDim + 64, y);
         }
         ++q_issued;
         KvIter itr = make_iter<BK, kCache>(p, u, s_cb, s_ib, s_pb);
@@ -339,15 +345,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if (!more) break;
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_empty(ks), ((kit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-          mbar_arrive_expect_tx(b_k_full(ks), C::kKVBytes);
-          tma_load_2d(sK + ks * C::kKVBytes, &p.tm_k, b_k_full(ks), u.g * kHeadDim, (int32_t)y);
-          tma_load_2d(sK + ks * C::kKVBytes + C::kSlabKV, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, (int32_t)y);
+          mbar_arrive_expect_tx(b_k_full(ks), C::kKBytes);
+          tma_load_2d(sK + ks * C::kKBytes, &p.tm_k, b_k_full(ks), u.g * kHeadDim, (int32_t)y);
+          if constexpr (!kFp8)
+            tma_load_2d(sK + ks * C::kKBytes + C::kSlabK, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, (int32_t)y);
           ++kit;
           const int vs = vit % C::kStages;
           if (!mbar_wait(b_v_empty(vs), ((vit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-          mbar_arrive_expect_tx(b_v_full(vs), C::kKVBytes);
-          tma_load_2d(sV + vs * C::kKVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, (int32_t)y);
-          tma_load_2d(sV + vs * C::kKVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, (int32_t)y);
+          mbar_arrive_expect_tx(b_v_full(vs), C::kVBytes);
+          tma_load_2d(sV + vs * C::kVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, (int32_t)y);
+          tma_load_2d(sV + vs * C::kVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, (int32_t)y);
           ++vit;
           if (*s_abort) { fail = true; break; }
         }
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const int vs = vit % C::kStages;
         if (!mbar_wait(b_v_full(vs), (vit / C::kStages) & 1, p.wait_limit_ns)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + vs * C::kKVBytes;
+        const uint32_t vbase = sV + vs * C::kVBytes;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSlabKV, 1024);
@@ -391,12 +398,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // S_k = Q_k K^T for the current item (K tile at kbase)
       auto qk = [&](int k, uint32_t kbase) {
         const uint32_t qbase = sQ + k * C::kQBytes;
+        if constexpr (kFp8) {
+          // 4 steps of 32 e4m3 = 32 bytes inside the single 128-byte swizzle atom
 #pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
-          const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * C::kSlabQ + koff, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * C::kSlabKV + koff, 16, 1024);
-          mma_ss(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kHeadDim / 32; ++kk) {
+            const uint64_t adesc = sdesc_sw128(qbase + kk * 32, 16, 1024);
+            const uint64_t bdesc = sdesc_sw128(kbase + kk * 32, 16, 1024);
+            mma_ss_f8(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+            const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
+            const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * C::kSlabQ + koff, 16, 1024);
+            const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * C::kSlabK + koff, 16, 1024);
+            mma_ss(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit(b_s_full0 + 8 * k);
         ++cnt[k];
@@ -421,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_full(ks), (kit / C::kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
-          const uint32_t kbase = sK + ks * C::kKVBytes;
+          const uint32_t kbase = sK + ks * C::kKBytes;
           if (n > 0 && !pv(0, n == 1)) { fail = true; break; }
           qk(0, kbase);
           if (u.nslot == 2) {
@@ -705,23 +722,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int BK, bool kCache>
+template <int BK, bool kCache, bool kFp8>
 static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<BK, kCache>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<BK>::kSmemMax);
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<BK, kCache, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<BK, kFp8>::kSmemMax);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  attn_kernel<BK, kCache><<<grid, kThreads, Cfg<BK>::smem_bytes(p.seq.num_seqs), st>>>(p);
+  attn_kernel<BK, kCache, kFp8><<<grid, kThreads, Cfg<BK, kFp8>::smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st) {
   const bool cache = p.seq.prefix_lens != nullptr || p.seq.block_table != nullptr;
-  if (p.seq.block == 128) return cache ? launch_attn_t<128, true>(p, grid, st) : launch_attn_t<128, false>(p, grid, st);
-  return cache ? launch_attn_t<64, true>(p, grid, st) : launch_attn_t<64, false>(p, grid, st);
+  if (p.fp8) {  // e4m3 Q / K: plain prefill only
+    if (cache) return cudaErrorNotSupported;
+    return p.seq.block == 128 ? launch_attn_t<128, false, true>(p, grid, st) : launch_attn_t<64, false, true>(p, grid, st);
+  }
+  if (p.seq.block == 128)
+    return cache ? launch_attn_t<128, true, false>(p, grid, st) : launch_attn_t<128, false, false>(p, grid, st);
+  return cache ? launch_attn_t<64, true, false>(p, grid, st) : launch_attn_t<64, false, false>(p, grid, st);
 }
 
 }  // namespace fp

@@ -83,6 +83,7 @@ struct __align__(64) AttnParams {
   int32_t* dev_status;
   uint64_t wait_limit_ns;
   int32_t test_unsignalled_wait;  // test hook: softmax warps first wait on a barrier nothing signals
+  int32_t fp8;                    // 1: tm_q / tm_k are e4m3 (uint8) maps, box {128, rows}; scales folded into scale_log2
 };
 
 constexpr int kMaxSeqs = FP_MAX_SEQS;
@@ -95,6 +96,8 @@ fp_status set_error(fp_status st, const char* fmt, ...);
 cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st);
 cudaError_t launch_search(const SearchParams& p, cudaStream_t st);
 cudaError_t launch_validate(const ValidateParams& p, cudaStream_t st);
+// Cumulative top-p selection (comparison selector): scores scratch [index_elems] floats.
+cudaError_t launch_topp(const SearchParams& p, float gamma, float* scores, cudaStream_t st);
 cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, long long n, cudaStream_t st);
 

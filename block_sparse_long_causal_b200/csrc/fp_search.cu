@@ -587,6 +587,236 @@ cudaError_t launch_search(const SearchParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// --------------------------------------------------------------------- top-p (comparison) ----
+// The cumulative-probability selector the max-based threshold replaces (FlashPrefill skill summary
+// page, "The Problem": Top-k / Top-p need score computation, sorting and cumulative sums;
+// FlexPrefill abstract, "Cumulative-Attention Based Index Selection"). Built to measure its cost
+// on the same pooled tensors: row (h, i) keeps block j iff the probability mass of the blocks that
+// are strictly more probable than j is below gamma (ties at the cut kept together), plus the sink
+// and the diagonal. It needs every score of a row before any decision, so it runs in two launches:
+// 1. topp_score_kernel writes the exact fp32 pooled scores into a scratch buffer laid out like the
+//    index lists (the score matrix the threshold search never materialises);
+// 2. topp_select_kernel, one warp per row: the row max, e_j = exp(s_j - max) and Z = sum e_j; then
+//    the cut x* = the smallest float x with F(x) = sum_{e_l > x} e_l < gamma * Z, found by
+//    bisection on the float bits (F is non-increasing, 0 <= e <= 1); block j is kept iff e_j >= x*
+//    (equivalently F(e_j) < gamma * Z); ascending emission with ballot/popc.
+__global__ void __launch_bounds__(kSearchThreads, 2) topp_score_kernel(const SearchParams p, float* scores) {
+  extern __shared__ __align__(16) unsigned char search_smem_raw[];
+  SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
+  const int S = p.seq.num_seqs;
+  int* t_cu = reinterpret_cast<int*>(search_smem_raw + sizeof(SearchSmem));
+  int* t_cb = t_cu + (S + 1);
+  int* t_ct = t_cb + (S + 1);
+  int* t_pb = t_ct + (S + 1);
+  int* t_ckb = t_pb + (S + 1);
+  long long* t_ib = reinterpret_cast<long long*>(((uintptr_t)(t_ckb + (S + 1)) + 7) & ~(uintptr_t)7);
+  if (!build_seq_tables(p.seq, t_cu, t_cb, t_ct, t_ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
+                        p.dev_status, t_pb, t_ckb))
+    return;
+  if (t_ib[S] != p.index_elems) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
+    return;
+  }
+  const int G = p.group, TI = p.rows_blocks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = t_ct[S];
+  for (int kr = 0;; ++kr) {
+    const int tile = kr * gridDim.x + ((kr & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+    if (tile >= num_tiles) break;
+    const int s = find_seq(t_ct, S, tile);
+    const int local = tile - t_ct[s];
+    const int nb = t_cb[s + 1] - t_cb[s];
+    const int ntiles = (nb + TI - 1) / TI;
+    const int it = ntiles - 1 - local / p.hkv;
+    const int g = local % p.hkv;
+    const int i0 = it * TI;
+    const int i_last = min(i0 + TI, nb) - 1;
+    const int gb0 = t_cb[s], pb = t_pb[s], kb0 = t_ckb[s];
+    const int jmax = pb + i_last;
+    const int nchunks = jmax / kKChunk + 1;
+    __syncthreads();  // previous tile done with shared memory
+    for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
+      const int r = e % kSearchRows, d4 = e / kSearchRows;
+      const int i = i0 + r / G;
+      const bool ok = r < TI * G && i <= i_last;
+      const float4 v = ok ? reinterpret_cast<const float4*>(
+                                p.q_pool + ((long long)(gb0 + i) * p.hq + g * G + r % G) * kHeadDim)[d4]
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      sm.qT[4 * d4 + 0][r] = v.x;
+      sm.qT[4 * d4 + 1][r] = v.y;
+      sm.qT[4 * d4 + 2][r] = v.z;
+      sm.qT[4 * d4 + 3][r] = v.w;
+    }
+    // this lane's rows 2*lane + e: list start and last key block (-1: padding row)
+    int64_t rbase[2];
+    int rj[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      const int i = i0 + r / G;
+      const bool ok = r < TI * G && i <= i_last;
+      rj[e] = ok ? pb + i : -1;
+      rbase[e] = ok ? list_row(t_cb, t_ib, t_pb, s, g * G + r % G, i) : 0;
+    }
+    issue_k_chunk(sm, 0, p.k_pool, kb0, g, p.hkv, 0, jmax);
+    for (int c = 0; c < nchunks; ++c) {
+      const int j0 = c * kKChunk;
+      if (c + 1 < nchunks) {
+        __syncthreads();  // buffer (c+1)&1 no longer read
+        issue_k_chunk(sm, (c + 1) & 1, p.k_pool, kb0, g, p.hkv, j0 + kKChunk, jmax);
+        cp_async_wait_all_but_one();
+      } else {
+        cp_async_wait_all();
+      }
+      __syncthreads();
+      float acc[2][8];
+      chunk_scores(sm, c & 1, warp, lane, acc);
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          const int j = j0 + 8 * warp + b;
+          if (j <= rj[e]) scores[rbase[e] + j] = acc[e][b] * p.inv_sqrt_d;
+        }
+    }
+  }
+}
+
+struct ToppParams {
+  SeqInfo seq;
+  int32_t hq;
+  float gamma;
+  const float* scores;   // row (s, h, i) at the index-list row start, pb + i + 1 entries
+  int32_t* counts;       // [Hq, NB]
+  int32_t* indices;
+  int64_t index_elems;
+  int32_t* dev_status;
+};
+
+constexpr int kToppPer = 32;  // scores per lane held in registers (rows of up to 1024 blocks)
+
+// F(x) = sum of e_l > x over the row (warp-wide), e in registers or re-read from the scratch
+__device__ __forceinline__ float topp_mass_above(const float (&e)[kToppPer], bool in_regs, const float* srow, float m,
+                                                 int n, float x) {
+  const int lane = threadIdx.x & 31;
+  float a = 0.f;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kToppPer; ++k) a += e[k] > x ? e[k] : 0.f;
+  } else {
+    for (int j = lane; j < n; j += 32) {
+      const float v = exp2f((srow[j] - m) * 1.4426950408889634f);
+      a += v > x ? v : 0.f;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return a;
+}
+
+__global__ void __launch_bounds__(256) topp_select_kernel(const ToppParams p) {
+  extern __shared__ int topp_tab[];
+  const int S = p.seq.num_seqs;
+  int* s_cu = topp_tab;
+  int* s_cb = s_cu + (S + 1);
+  int* s_pb = s_cb + (S + 1);
+  int* s_ckb = s_pb + (S + 1);
+  int* s_ok = s_ckb + (S + 1);
+  long long* s_ib = reinterpret_cast<long long*>(((uintptr_t)(s_ok + 1) + 7) & ~(uintptr_t)7);
+  if (!build_seq_tables(p.seq, s_cu, s_cb, nullptr, s_ib, p.hq, 0, 0, s_ok, p.dev_status, s_pb, s_ckb)) return;
+  if (s_ib[S] != p.index_elems) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const long long rows = (long long)p.hq * p.seq.total_blocks;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows; w += warps) {
+    const int h = (int)(w / p.seq.total_blocks), gb = (int)(w % p.seq.total_blocks);
+    const int s = find_seq(s_cb, S, gb);
+    const int i = gb - s_cb[s];
+    const int jd = s_pb[s] + i, n = jd + 1;
+    const int64_t base = list_row(s_cb, s_ib, s_pb, s, h, i);
+    const float* srow = p.scores + base;
+    const bool in_regs = n <= 32 * kToppPer;
+    float m = -INFINITY;
+    for (int j = lane; j < n; j += 32) m = fmaxf(m, srow[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float e[kToppPer];
+    float z = 0.f;
+#pragma unroll
+    for (int k = 0; k < kToppPer; ++k) {
+      const int j = lane + 32 * k;
+      e[k] = (in_regs && j < n) ? exp2f((srow[j] - m) * 1.4426950408889634f) : 0.f;
+      z += e[k];
+    }
+    if (!in_regs)
+      for (int j = lane; j < n; j += 32) z += exp2f((srow[j] - m) * 1.4426950408889634f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    // the cut x*: keep j iff e_j >= x*  (x* = 0 keeps all, x* above 1 keeps none but the forced)
+    uint32_t cut;
+    if (p.gamma >= 1.f) {
+      cut = 0u;
+    } else if (!(p.gamma > 0.f)) {
+      cut = 0x7f800000u;  // +inf
+    } else {
+      const float gz = p.gamma * z;
+      uint32_t lo = 0u, hi = 0x3f800000u;  // F(1.0) = 0 < gamma * z
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (topp_mass_above(e, in_regs, srow, m, n, __uint_as_float(mid)) < gz) hi = mid; else lo = mid + 1u;
+      }
+      cut = lo;
+    }
+    const float xcut = __uint_as_float(cut);
+    int cnt = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      float v = 0.f;
+      if (j < n) v = exp2f((srow[j] - m) * 1.4426950408889634f);
+      const bool keep = j < n && (j == 0 || j == jd || v >= xcut);
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if (keep) p.indices[base + cnt + __popc(bal & lt_mask)] = j;
+      cnt += __popc(bal);
+    }
+    if (lane == 0) p.counts[(long long)h * p.seq.total_blocks + gb] = cnt;
+  }
+}
+
+cudaError_t launch_topp(const SearchParams& sp, float gamma, float* scores, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(topp_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)search_smem_bytes(kMaxSeqs));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int cap = 2 * sms;
+  const int grid = sp.num_tiles < cap ? sp.num_tiles : cap;
+  if (grid <= 0) return cudaSuccess;
+  topp_score_kernel<<<grid, kSearchThreads, (int)search_smem_bytes(sp.seq.num_seqs), st>>>(sp, scores);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ToppParams tp;
+  tp.seq = sp.seq;
+  tp.hq = sp.hq;
+  tp.gamma = gamma;
+  tp.scores = scores;
+  tp.counts = sp.counts;
+  tp.indices = sp.indices;
+  tp.index_elems = sp.index_elems;
+  tp.dev_status = sp.dev_status;
+  const size_t tab = (size_t)(4 * (sp.seq.num_seqs + 1) + 1) * 4 + 8 + (size_t)(sp.seq.num_seqs + 1) * 8;
+  topp_select_kernel<<<sms * 8, 256, tab, st>>>(tp);
+  return cudaGetLastError();
+}
+
 // -------------------------------------------------------------------------------- validate ----
 // One warp per list row (s, h, i), with jd = pb + i the row's diagonal key block: count in
 // [1, jd+1]; entries ascending, in [0, jd]; first 0; last jd.

@@ -107,6 +107,19 @@ FP_API fp_status fp_block_pool(const fp_problem* p, const void* q, const void* k
 FP_API fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
                           int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream);
 
+/* Comparison selector (not the method: the one its threshold replaces). Cumulative top-p block
+ * selection on the same pooled scores (FlashPrefill skill summary page, "The Problem": Top-k /
+ * Top-p need score computation, sorting and cumulative sums; FlexPrefill abstract,
+ * "Cumulative-Attention Based Index Selection"): row (h, i) keeps block j iff the softmax mass of
+ * the blocks strictly more probable than j is below gamma (blocks tied at the cut together), plus
+ * j = 0 and j = i. gamma <= 0 keeps those two only, gamma >= 1 every causal block; gamma finite.
+ * It needs a whole row of scores before any decision: scores is a device float32 scratch of
+ * index_elems entries (the pooled score matrix, laid out like the index lists) written and read
+ * by the call. counts / indices as for fp_block_search. */
+FP_API fp_status fp_block_search_topp(const fp_problem* p, const float* q_pool, const float* k_pool, float gamma,
+                                      float* scores, int32_t* counts, int32_t* indices, int32_t* dev_status,
+                                      void* stream);
+
 /* Steps 1 + 2 in one call: fp_block_pool followed by fp_block_search on the same stream (two
  * launches: Q and K are streamed once by the pool kernel at HBM bandwidth; the search kernel
  * then computes the block scores, the threshold and the lists without materialising scores).
@@ -128,6 +141,24 @@ FP_API fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const 
 /* Dense causal attention (every causal block), same kernel design; the baseline for the speedup. */
 FP_API fp_status fp_dense_attn(const fp_problem* p, const void* q, const void* k, const void* v, float softmax_scale,
                         void* out, float* lse, int32_t* dev_status, void* stream);
+
+/* FP8 attention (FlashPrefill V2 abstract: FP8 inference). Q and K hold e4m3 codes (OCP E4M3, one
+ * byte per element, row-major [tokens, heads, head_dim], dequantised value = q_scale * code value,
+ * resp. k_scale; per-tensor scales, finite and positive); V, P and O stay bf16. Q K^T runs on the
+ * tensor cores in e4m3 (tcgen05 kind::f8f6f4) with fp32 accumulation; the logits are
+ * softmax_scale * q_scale * k_scale * (q . k), softmax_scale <= 0 selecting 1/sqrt(d).
+ * counts / indices / out / lse / dev_status as for fp_block_sparse_attn (lists from any search,
+ * e.g. fp_block_search on the bf16 Q and K the e4m3 codes were quantised from). Plain prefill
+ * only (no paged-cache variant). */
+FP_API fp_status fp_block_sparse_attn_fp8(const fp_problem* p, const void* q_e4m3, const void* k_e4m3, const void* v,
+                                          float q_scale, float k_scale, const int32_t* counts, const int32_t* indices,
+                                          float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                                          void* stream);
+
+/* Dense causal FP8 attention (every causal block), the FP8 baseline. */
+FP_API fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q_e4m3, const void* k_e4m3, const void* v,
+                                   float q_scale, float k_scale, float softmax_scale, void* out, float* lse,
+                                   int32_t* dev_status, void* stream);
 
 /* Bytes of workspace fp_sparse_prefill needs for this problem: the pooled Q and K, the counts and
  * the index lists, each 256-byte aligned. */

@@ -94,6 +94,38 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+# ---- FP8 e4m3 (OCP "E4M3": 1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinity,
+# 0x7F / 0xFF are NaN; largest finite 448). Input-format conversion for the FP8 attention inputs.
+def _e4m3_table() -> np.ndarray:
+    """Values of the codes 0x00..0x7E (the non-negative finite e4m3 numbers), ascending."""
+    vals = []
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        vals.append((m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(vals, np.float64)
+
+
+_E4M3 = _e4m3_table()
+
+
+def to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """float -> e4m3 codes (uint8): round to nearest, ties to the even code, saturate to +-448."""
+    x = np.asarray(x, np.float64)
+    a = np.minimum(np.abs(x), _E4M3[-1])
+    hi = np.clip(np.searchsorted(_E4M3, a, side="left"), 0, len(_E4M3) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - _E4M3[lo], _E4M3[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(x), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def e4m3_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    b = np.asarray(b, np.uint8)
+    v = _E4M3[np.minimum(b & 0x7F, 0x7E)].astype(np.float32)
+    return np.where(b & 0x80, -v, v).astype(np.float32)
+
+
 def _pool():
     return _cf.ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1)))
 

@@ -182,3 +182,23 @@ def test_paged_calls_check_the_cache_and_arguments():
     # a hand-edited cache inconsistent with the problem
     c.page_size = 100
     assert fp._lib.fp_paged_block_pool(C.byref(p), C.byref(c), ok, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
+
+
+def test_fp8_calls_reject_bad_scales_before_launch():
+    st, p = _prob()
+    ok = C.c_void_p(4096)
+    for qs, ks in ((0.0, 1.0), (1.0, -2.0), (float("nan"), 1.0), (1.0, float("inf")), (1e30, 1e30)):
+        assert fp._lib.fp_block_sparse_attn_fp8(C.byref(p), ok, ok, ok, C.c_float(qs), C.c_float(ks), ok, ok,
+                                                C.c_float(0.0), ok, None, None, None) == fp.FP_ERR_INVALID_ARG
+        assert fp._lib.fp_dense_attn_fp8(C.byref(p), ok, ok, ok, C.c_float(qs), C.c_float(ks), C.c_float(0.0), ok,
+                                         None, None, None) == fp.FP_ERR_INVALID_ARG
+    assert "scale" in _err()
+
+
+def test_topp_rejects_bad_arguments_before_launch():
+    st, p = _prob()
+    ok = C.c_void_p(4096)
+    assert fp._lib.fp_block_search_topp(C.byref(p), ok, ok, C.c_float(float("nan")), ok, ok, ok, None,
+                                        None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_block_search_topp(C.byref(p), ok, ok, C.c_float(0.9), None, ok, ok, None,
+                                        None) == fp.FP_ERR_INVALID_ARG
