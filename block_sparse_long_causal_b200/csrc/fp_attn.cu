@@ -36,6 +36,11 @@
 // the K/V of one kv-head (L2 resident) and the longest causal rows start first.
 // Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, lets issued copies and MMAs
 // finish, frees TMEM and returns.
+// Instances (template flags): kCache -- chunked prefill onto a (paged) K/V cache: each K/V block's
+// TMA row comes from the block table and a query's causal limit is its key position (cached prefix
+// + local position); the plain prefill is compiled without it. kFp8 -- e4m3 Q and K: their tiles
+// are single 128-byte-row slabs loaded as uint8 boxes and Q K^T runs as kind::f8f6f4 (K = 32 per
+// MMA); V, P and O stay bf16 and the per-tensor scales are folded into the softmax scale.
 #include "fp_internal.h"
 #include "fp_seq.cuh"
 
