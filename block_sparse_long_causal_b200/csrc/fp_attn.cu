@@ -29,7 +29,8 @@
 //   G odd:           one q-head, query tiles (2m+1, 2m) (the last may run alone).
 // The kv iteration is the ascending union of the slots' lists (two per slot when B = 64, where a
 // 128-row tile holds two query blocks); a per-(slot, half) bit masks rows whose list lacks the
-// current block, so different lists stay exact.
+// current block, so different lists stay exact, and a slot none of whose lists holds the block
+// skips the item altogether (no QK, PV or softmax for it).
 // Because QK_k(n) is issued after PV_k(n-1) and tcgen05.commit tracks all earlier MMAs, a slot
 // that sees S_k(n) may rescale O_k without waiting: PV_k(n-1) has already completed.
 // Units are ordered kv-head outermost, then by descending query tile, so concurrent CTAs stream
@@ -436,26 +437,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
         if (!mbar_wait(b_q_full, uc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
+        // Only the slots whose lists hold an item's block take part in it (bits 2k, 2k+1 of its
+        // row mask): the others skip its QK, PV and softmax. A slot's PV for item n-1 is issued at
+        // item n (before its QK of item n, whose S overwrites P), so V(n-1) is released there.
         int e, n = 0;
+        int prev_part = 0;          // slots that took part in the previous item (their PV is due)
+        bool had_pv[2] = {false, false};
         if (!read_item(e)) { fail = true; break; }
         bool more = e != kItemEnd;
         while (more) {
+          const int mask = e & 15;
+          const int part = (((mask & 3) != 0) ? 1 : 0) | (((mask & 12) != 0 && u.nslot == 2) ? 2 : 0);
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_full(ks), (kit / C::kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
           const uint32_t kbase = sK + ks * C::kKBytes;
-          if (n > 0 && !pv(0, n == 1)) { fail = true; break; }
-          qk(0, kbase);
-          if (u.nslot == 2) {
-            if (n > 0 && !pv(1, n == 1)) { fail = true; break; }
-            qk(1, kbase);
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            if ((prev_part >> sl) & 1) {
+              if (!pv(sl, !had_pv[sl])) { fail = true; break; }
+              had_pv[sl] = true;
+            }
+            if ((part >> sl) & 1) qk(sl, kbase);
           }
-          if (n > 0) {  // both PVs of the previous item are issued: release its V tile
+          if (fail) break;
+          if (n > 0) {  // the previous item's PVs are issued: release its V tile
             mma_commit(b_v_empty(vit % C::kStages));
             ++vit;
           }
           mma_commit(b_k_empty(ks));
           ++kit;
+          prev_part = part;
           if (!read_item(e)) { fail = true; break; }
           more = e != kItemEnd;
           if (!more) mma_commit(b_q_empty);
@@ -464,12 +476,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         if (fail) break;
         if (n > 0) {
-          if (!pv(0, n == 1)) { fail = true; break; }
-          if (u.nslot == 2 && !pv(1, n == 1)) { fail = true; break; }
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            if ((prev_part >> sl) & 1) {
+              if (!pv(sl, !had_pv[sl])) { fail = true; break; }
+              had_pv[sl] = true;
+            }
+          }
+          if (fail) break;
           mma_commit(b_v_empty(vit % C::kStages));
           ++vit;
-          mma_commit(b_o_final0);
-          if (u.nslot == 2) mma_commit(b_o_final0 + 8);
+          if (had_pv[0]) mma_commit(b_o_final0);
+          if (had_pv[1]) mma_commit(b_o_final0 + 8);
         } else {
           mma_commit(b_q_empty);  // empty kv list: release Q without touching O
         }
@@ -520,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (e == kItemEnd) break;
         if (!active) continue;
         const int j = e >> 4, mask = e & 15;
+        if (((mask >> (2 * slot)) & 3) == 0) continue;  // no list of this slot holds block j
         // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
         if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
