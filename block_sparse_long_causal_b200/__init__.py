@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(_HERE, "libfp.so")
 FP_OK, FP_ERR_INVALID_ARG, FP_ERR_UNSUPPORTED, FP_ERR_CUDA, FP_ERR_TIMEOUT = 0, 1, 2, 3, 4
 FP_DEV_TIMEOUT, FP_DEV_BAD_LIST, FP_DEV_BAD_PROBLEM = 1, 2, 4
 FP_MAX_SEQS = 1024
+FP_SCHED_WORDS = 2  # int32 words of the attention work counter (fp_problem.sched)
 FP_NOALLOC_MAX_BYTES = 64 << 20
 EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_pool_search", "fp_block_sparse_attn",
             "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill", "fp_sparse_prefill_noalloc",
@@ -52,7 +53,7 @@ class fp_problem(C.Structure):
     _fields_ = [("cu_seqlens", C.c_void_p), ("num_seqs", C.c_int32), ("total_tokens", C.c_int32),
                 ("total_blocks", C.c_int32), ("max_seq_blocks", C.c_int32), ("index_elems", C.c_int64),
                 ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
-                ("block_size", C.c_int32)]
+                ("block_size", C.c_int32), ("sched", C.c_void_p)]
 
 
 class fp_paged_cache(C.Structure):
@@ -132,10 +133,13 @@ def _stream(stream):
 
 
 class Problem:
-    """fp_problem plus the device cu_seqlens tensor it points to (kept alive here)."""
+    """fp_problem plus the device tensors it points to (kept alive here): cu_seqlens and, with
+    work_counter (the default on a CUDA device), the attention calls' work counter -- zeroed once,
+    left at zero by every launch, so launches of this problem must be ordered (one stream, or
+    events); give concurrent streams one Problem each."""
 
     def __init__(self, cu_seqlens_host, cu_seqlens_dev: torch.Tensor, num_q_heads: int, num_kv_heads: int,
-                 head_dim: int, block_size: int):
+                 head_dim: int, block_size: int, work_counter: bool = True):
         host = np.ascontiguousarray(cu_seqlens_host, np.int32)
         if cu_seqlens_dev.dtype != torch.int32:
             raise ValueError("cu_seqlens must be int32")
@@ -144,6 +148,10 @@ class Problem:
         self.c = fp_problem()
         _check(_lib.fp_problem_init(C.byref(self.c), host.ctypes.data_as(C.c_void_p), len(host) - 1,
                                     _ptr(cu_seqlens_dev), num_q_heads, num_kv_heads, head_dim, block_size))
+        self.sched = None
+        if work_counter and cu_seqlens_dev.is_cuda:
+            self.sched = torch.zeros(FP_SCHED_WORDS, dtype=torch.int32, device=cu_seqlens_dev.device)
+            self.c.sched = self.sched.data_ptr()
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)
@@ -154,10 +162,10 @@ class Problem:
 
 
 def problem(cu_seqlens_host, num_q_heads: int, num_kv_heads: int, head_dim: int = 128, block_size: int = 128,
-            device="cuda") -> Problem:
+            device="cuda", work_counter: bool = True) -> Problem:
     host = np.ascontiguousarray(cu_seqlens_host, np.int32)
     dev = torch.from_numpy(host.copy()).to(device)
-    return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size)
+    return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size, work_counter)
 
 
 def block_pool(p: Problem, q, k, q_pool, k_pool, stream=None):

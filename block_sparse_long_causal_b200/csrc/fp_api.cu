@@ -142,6 +142,7 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(FP_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
   if (!std::isfinite(softmax_scale)) return fail(FP_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if ((reinterpret_cast<uintptr_t>(p->sched) & 3u) != 0) return fail(FP_ERR_INVALID_ARG, "problem.sched must be 4-byte aligned");
   if (p->total_tokens == 0) return FP_OK;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)p->head_dim);
 
@@ -166,6 +167,7 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   a.index_elems = index_elems(p, c);
   a.scale_log2 = scale * qk_scale * 1.4426950408889634f;
   a.fp8 = fp8 ? 1 : 0;
+  a.sched = p->sched;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.dev_status = dev_status;
@@ -367,7 +369,7 @@ fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q, const void* k, c
 
 namespace {
 struct WorkspaceLayout {
-  int64_t q_pool, k_pool, counts, indices, total;  // byte offsets and total size
+  int64_t q_pool, k_pool, counts, indices, sched, total;  // byte offsets and total size
 };
 int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
 WorkspaceLayout workspace_layout(const fp_problem* p) {
@@ -377,7 +379,8 @@ WorkspaceLayout workspace_layout(const fp_problem* p) {
   w.k_pool = align256(w.q_pool + nb * p->num_q_heads * d * 4);
   w.counts = align256(w.k_pool + nb * p->num_kv_heads * d * 4);
   w.indices = align256(w.counts + (int64_t)p->num_q_heads * nb * 4);
-  w.total = align256(w.indices + p->index_elems * 4);
+  w.sched = align256(w.indices + p->index_elems * 4);
+  w.total = align256(w.sched + FP_SCHED_WORDS * 4);
   return w;
 }
 }  // namespace
@@ -406,9 +409,15 @@ fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, c
   float* k_pool = reinterpret_cast<float*>(base + w.k_pool);
   int32_t* counts = reinterpret_cast<int32_t*>(base + w.counts);
   int32_t* indices = reinterpret_cast<int32_t*>(base + w.indices);
+  // the work counter lives in the workspace (scratch between calls): zeroed here, in stream order
+  fp_problem pw = *p;
+  pw.sched = reinterpret_cast<int32_t*>(base + w.sched);
+  if ((st = cuda_status(cudaMemsetAsync(pw.sched, 0, FP_SCHED_WORDS * sizeof(int32_t),
+                                        static_cast<cudaStream_t>(stream)), "work counter reset")) != FP_OK)
+    return st;
   if ((st = fp_block_pool(p, q, k, q_pool, k_pool, stream)) != FP_OK) return st;
   if ((st = fp_block_search(p, q_pool, k_pool, tau, counts, indices, dev_status, stream)) != FP_OK) return st;
-  return fp_block_sparse_attn(p, q, k, v, counts, indices, softmax_scale, out, lse, dev_status, stream);
+  return fp_block_sparse_attn(&pw, q, k, v, counts, indices, softmax_scale, out, lse, dev_status, stream);
 }
 
 namespace {
@@ -523,6 +532,6 @@ fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t
 
 const char* fp_last_error(void) { return g_err; }
 
-int32_t fp_version(void) { return 200; }
+int32_t fp_version(void) { return 201; }
 
 }  // extern "C"

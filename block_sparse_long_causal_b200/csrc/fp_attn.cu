@@ -34,7 +34,10 @@
 // Because QK_k(n) is issued after PV_k(n-1) and tcgen05.commit tracks all earlier MMAs, a slot
 // that sees S_k(n) may rescale O_k without waiting: PV_k(n-1) has already completed.
 // Units are ordered kv-head outermost, then by descending query tile, so concurrent CTAs stream
-// the K/V of one kv-head (L2 resident) and the longest causal rows start first.
+// the K/V of one kv-head (L2 resident) and the longest causal rows start first. With a work counter
+// (fp_problem.sched) each CTA takes the next untaken unit of that order when its producer is free,
+// which keeps the grid balanced for lists of any lengths (a fixed share per CTA left the busiest
+// SM 4-15% above the mean on the 128K workload, more the sparser the lists).
 // Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, lets issued copies and MMAs
 // finish, frees TMEM and returns.
 // Instances (template flags): kCache -- chunked prefill onto a (paged) K/V cache: each K/V block's
@@ -61,14 +64,15 @@ static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * 168,
 constexpr unsigned kPolyPairs = 0x00u;
 // Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
-// Item ring: the producer merges the index lists once and publishes each kv item as
-// (block << 4 | row-mask bits) in a shared ring, one mbarrier per entry; -1 ends a unit. The
-// producer can never lead the slowest reader by more than 2 * (kStages + 3) entries (a K load waits for
-// the QK of item n - kStages, which needs both slots' P of the item before), so the ring keeps a
-// parity wait from ever seeing a phase two ahead (32 leaves room for one-item units, which add an
-// end marker per item).
+// Item ring: the producer merges the index lists once and publishes, per unit, the unit's index,
+// then each kv item as (block << 4 | row-mask bits), then kItemEnd; after its last unit, kUnitsEnd.
+// Each entry has a full and an empty mbarrier: the MMA thread and every softmax warp arrive on the
+// empty barrier once they have read the entry, and the producer waits on it before writing the
+// entry's next use, so no reader can be overrun however far it lags.
 constexpr int kRing = 32;
+constexpr int kRingReaders = 9;  // the MMA thread and the 8 softmax warps
 constexpr int kItemEnd = -1;
+constexpr int kUnitsEnd = -2;
 // Largest row sum of one item that the fast path (no max pass) accepts; see the softmax loop.
 constexpr float kFastSumLimit = 65536.f;
 
@@ -92,8 +96,9 @@ struct Cfg {
   static constexpr uint32_t kOffV = kOffK + kStages * kKBytes;
   static constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
   // barriers: q_full, q_empty, k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2],
-  // o_final[2], drain, never (the test hook's barrier that nothing arrives on), item[kRing]
-  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2 + kRing;
+  // o_final[2], drain, never (the test hook's barrier that nothing arrives on), item_full[kRing],
+  // item_empty[kRing]
+  static constexpr int kNumBars = 2 + 4 * kStages + 6 + 2 + 2 * kRing;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag, ok
   static constexpr uint32_t kOffRing = kOffMisc + 16;               // kRing int32 item entries
   static constexpr uint32_t kOffTab = (kOffRing + 4 * kRing + 15) & ~15u;
@@ -161,10 +166,28 @@ __device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s
   return u;
 }
 
-// k-th unit of this CTA in a boustrophedon order over the grid (balances the descending sizes).
+// Unit schedule. Every CTA starts with unit blockIdx.x. With a work counter (p.sched) each further
+// unit is the next one in the global order that no CTA has taken yet (greedy: a CTA that finishes
+// early takes more, so the grid ends together whatever the lists' lengths); without one, the k-th
+// unit of the CTA follows a boustrophedon order over the grid (balanced only for causal-dense sizes).
+// The global order keeps the CTAs on neighbouring units either way: one kv-head's K/V at a time.
 __device__ __forceinline__ int unit_of(int k) {
   const int g = gridDim.x;
   return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+__device__ __forceinline__ int next_unit(int* sched, int k) {
+  return sched ? (int)gridDim.x + atomicAdd(sched, 1) : unit_of(k);
+}
+// Called once per CTA after its last fetch: the grid's last CTA returns both counter words to zero
+// (no fetch of this launch can follow), so launches ordered on a stream share the counter.
+__device__ __forceinline__ void sched_release(int* sched) {
+  if (!sched) return;
+  __threadfence();
+  if (atomicAdd(sched + 1, 1) == (int)gridDim.x - 1) {
+    __threadfence();
+    atomicExch(sched, 0);
+    atomicExch(sched + 1, 0);
+  }
 }
 
 // ---------------------------------------------------------------------- kv iteration -----------
@@ -252,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const uint32_t b_o_final0 = b_p_full0 + 16;
   const uint32_t b_drain = b_o_final0 + 16, b_never = b_drain + 8;
   auto b_item = [&](uint32_t x) { return b_never + 8 + 8 * (x % kRing); };
+  auto b_item_empty = [&](uint32_t x) { return b_never + 8 + 8 * kRing + 8 * (x % kRing); };
   volatile int* s_item = reinterpret_cast<volatile int*>(smem + C::kOffRing);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -285,7 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     mbar_init(b_drain, 1);
     mbar_init(b_never, 1);
-    for (int i = 0; i < kRing; ++i) mbar_init(b_item(i), 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(b_item(i), 1);
+      mbar_init(b_item_empty(i), kRingReaders);
+    }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -321,10 +348,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       int uc = 0, q_issued = 0;   // units started / Q loads issued
       bool fail = false;
       bool bad_list = false, bad_page = false;
-      for (int k = 0;; ++k, ++uc) {
-        const int t = unit_of(k);
+      // write the next ring entry once every reader has read the one it replaces
+      auto publish = [&](int val) -> bool {
+        if (xit >= (uint32_t)kRing && !mbar_wait(b_item_empty(xit), ((xit / kRing) - 1) & 1, p.wait_limit_ns))
+          return false;
+        s_item[xit % kRing] = val;
+        mbar_arrive(b_item(xit));
+        ++xit;
+        return true;
+      };
+      int t = blockIdx.x;
+      for (int k = 0;; ++uc) {
         if (t >= num_units || fail) break;
         const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
+        if (!publish(t)) { fail = true; break; }
         if (!mbar_wait(b_q_empty, (uc & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
         mbar_arrive_expect_tx(b_q_full, C::kQBytes * u.nslot);
         for (int sl = 0; sl < u.nslot; ++sl) {
@@ -345,9 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
               more = itr.next(j, mask);
             }
           }
-          s_item[xit % kRing] = more ? (j << 4) | mask : kItemEnd;  // publish the item (or the unit's end)
-          mbar_arrive(b_item(xit));
-          ++xit;
+          if (!publish(more ? (j << 4) | mask : kItemEnd)) { fail = true; break; }  // the item, or the unit's end
           if (!more) break;
           const int ks = kit % C::kStages;
           if (!mbar_wait(b_k_empty(ks), ((kit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
@@ -365,7 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if (*s_abort) { fail = true; break; }
         }
         bad_list |= itr.bad;
+        if (!fail) t = next_unit(p.sched, ++k);
       }
+      if (!fail && !publish(kUnitsEnd)) fail = true;
+      sched_release(p.sched);
       if (bad_list) dev_flag(p.dev_status, kDevBadList);
       if (bad_page) dev_flag(p.dev_status, kDevBadProblem);
       if (fail) {
@@ -428,12 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       auto read_item = [&](int& e) -> bool {
         if (!mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns)) return false;
         e = s_item[xit % kRing];
+        mbar_arrive(b_item_empty(xit));
         ++xit;
         return true;
       };
-      for (int k = 0;; ++k, ++uc) {
-        const int t = unit_of(k);
-        if (t >= num_units || fail) break;
+      for (;; ++uc) {
+        int t;
+        if (!read_item(t)) { fail = true; break; }
+        if (t == kUnitsEnd) break;
         const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
         if (!mbar_wait(b_q_full, uc & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
@@ -519,9 +559,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     bool fail = false;
     if (p.test_unsignalled_wait && num_units > 0)
       fail = __any_sync(kFull, !mbar_wait(b_never, 0, p.wait_limit_ns));
-    for (int k = 0;; ++k) {
-      const int t = unit_of(k);
-      if (t >= num_units || fail) break;
+    // the next ring entry (warp-collective; lane 0 releases the entry once the whole warp has read it)
+    auto read_entry = [&](int& e) -> bool {
+      if (__any_sync(kFull, !mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns))) return false;
+      e = s_item[xit % kRing];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_item_empty(xit));
+      ++xit;
+      return true;
+    };
+    while (!fail) {
+      int t;
+      if (!read_entry(t)) { fail = true; break; }
+      if (t == kUnitsEnd) break;
       const Unit u = decode_unit(t, s_cu, s_cb, s_ct, s_pb, S, p.group);
       const bool active = slot < u.nslot;     // an idle slot only consumes the unit's ring entries
       const int qpos = u.qt[slot] * kTileM + r;  // local query position of this row
@@ -532,9 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       float m_run = -INFINITY, l_run = 0.f;
       int n = 0;
       while (true) {
-        if (__any_sync(kFull, !mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns))) { fail = true; break; }
-        const int e = s_item[xit % kRing];
-        ++xit;
+        int e;
+        if (!read_entry(e)) { fail = true; break; }
         if (e == kItemEnd) break;
         if (!active) continue;
         const int j = e >> 4, mask = e & 15;

@@ -83,7 +83,18 @@ typedef struct fp_problem {
   int32_t num_kv_heads;      /* Hkv */
   int32_t head_dim;          /* d; 128 is supported */
   int32_t block_size;        /* B; 64 or 128 */
+  int32_t* sched;            /* optional work counter of the attention calls, see below; NULL after init */
 } fp_problem;
+
+/* Work counter. fp_problem_init leaves sched NULL: an attention launch then gives each CTA a fixed
+ * share of the (q-head pair, 128-row query tile) units, balanced for causal-dense lists. A caller
+ * may point sched at FP_SCHED_WORDS device int32 that hold zero: each CTA then takes its next unit
+ * from the counter when it is free, so the work stays balanced whatever the lists' lengths. Every
+ * launch leaves the words at zero again, so the same words serve any number of launches (and CUDA
+ * graph replays) that run one after another; two launches that may run at the same time (other
+ * streams, no ordering between them) must not share them. The results are identical either way.
+ * fp_sparse_prefill(_noalloc) use words inside their workspace and ignore sched. */
+#define FP_SCHED_WORDS 2
 
 /* Fill *p from a HOST copy of cu_seqlens (read only during the call) and the device copy that the
  * kernels will read. Checks sizes and the sequence limits. */

@@ -112,7 +112,7 @@ def test_sparse_prefill_workspace_and_argument_checks():
     assert fp._lib.fp_sparse_prefill_workspace(C.byref(p), C.byref(n)) == fp.FP_OK
     nb = 3 + 1 + 4
     need = 0
-    for nbytes in (nb * 4 * 128 * 4, nb * 2 * 128 * 4, 4 * nb * 4, p.index_elems * 4):
+    for nbytes in (nb * 4 * 128 * 4, nb * 2 * 128 * 4, 4 * nb * 4, p.index_elems * 4, fp.FP_SCHED_WORDS * 4):
         need += (nbytes + 255) // 256 * 256
     assert n.value == need
     ok, null = C.c_void_p(4096), None
