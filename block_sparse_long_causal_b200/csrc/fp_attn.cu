@@ -36,8 +36,8 @@
 // Units are ordered kv-head outermost, then by descending query tile, so concurrent CTAs stream
 // the K/V of one kv-head (L2 resident) and the longest causal rows start first. With a work counter
 // (fp_problem.sched) each CTA takes the next untaken unit of that order when its producer is free,
-// which keeps the grid balanced for lists of any lengths (a fixed share per CTA left the busiest
-// SM 4-15% above the mean on the 128K workload, more the sparser the lists).
+// which keeps the grid balanced for lists of any lengths (a load model of the 128K workload puts
+// the busiest SM of a fixed share 4-15% above the mean, more the sparser the lists).
 // Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, lets issued copies and MMAs
 // finish, frees TMEM and returns.
 // Instances (template flags): kCache -- chunked prefill onto a (paged) K/V cache: each K/V block's
