@@ -270,20 +270,23 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert int(sp.dev_status.item()) == 0, "device status after warm-up"
 
-    # dense baseline (own kernel, same design) for the speedup, timed on the same inputs
+    # dense baseline (own kernel, same design) for the speedup, timed on the same inputs and the
+    # same way as the sparse attention in the step: after the pool + search call, one event pair
+    # around each launch
     dense_ms = None
     if not args.no_dense:
         for _ in range(2):
             fp.dense_attn(p, q, k, v, 0.0, sp.out, None, sp.dev_status, stream)
         torch.cuda.synchronize()
-        d0, d1 = ev(), ev()
         nd = max(1, min(3, args.steps))
-        d0.record(stream)
-        for _ in range(nd):
+        dev_ = [[ev(), ev()] for _ in range(nd)]
+        for e0, e1 in dev_:
+            fp.block_pool_search(p, q, k, tau, sp.q_pool, sp.k_pool, sp.counts, sp.indices, sp.dev_status, stream)
+            e0.record(stream)
             fp.dense_attn(p, q, k, v, 0.0, sp.out, None, sp.dev_status, stream)
-        d1.record(stream)
+            e1.record(stream)
         torch.cuda.synchronize()
-        dense_ms = d0.elapsed_time(d1) / nd
+        dense_ms = sum(e0.elapsed_time(e1) for e0, e1 in dev_) / nd
 
     supp = None if args.no_supplementary else supplementary(fp, p, sp, x, q, k, v, tau, stream, w)
 

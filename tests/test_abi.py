@@ -70,6 +70,19 @@ def test_problem_init_rejects_too_many_sequences():
     assert st == fp.FP_ERR_INVALID_ARG
 
 
+def test_work_counter_is_null_after_init_and_checked_for_alignment():
+    st, p = _prob()
+    assert st == fp.FP_OK and not p.sched
+    ok, null = C.c_void_p(4096), None
+    p.sched = 4098  # not 4-byte aligned: rejected on the host, before any launch
+    for dense in (False, True):
+        if dense:
+            r = fp._lib.fp_dense_attn(C.byref(p), ok, ok, ok, C.c_float(0), ok, null, null, null)
+        else:
+            r = fp._lib.fp_block_sparse_attn(C.byref(p), ok, ok, ok, ok, ok, C.c_float(0), ok, null, null, null)
+        assert r == fp.FP_ERR_INVALID_ARG and "sched" in _err()
+
+
 def test_empty_sequences_are_allowed():
     st, p = _prob(cu=(0, 0, 5, 5))
     assert st == fp.FP_OK and p.total_blocks == 1
