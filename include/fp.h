@@ -171,15 +171,16 @@ FP_API fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q_e4m3, cons
                                    float q_scale, float k_scale, float softmax_scale, void* out, float* lse,
                                    int32_t* dev_status, void* stream);
 
-/* Bytes of workspace fp_sparse_prefill needs for this problem: the pooled Q and K, the counts and
- * the index lists, each 256-byte aligned. */
+/* Bytes of workspace fp_sparse_prefill needs for this problem: the pooled Q and K, the counts, the
+ * index lists and the attention's work counter (FP_SCHED_WORDS int32), each 256-byte aligned. */
 FP_API fp_status fp_sparse_prefill_workspace(const fp_problem* p, int64_t* bytes);
 
 /* The whole sparse prefill in one call (FlashPrefill: block pooling, max-based block search and
  * block-sparse attention): fp_block_pool, fp_block_search and fp_block_sparse_attn on `stream`,
  * with the intermediate tensors in `workspace` (device, 256-byte aligned, at least
- * fp_sparse_prefill_workspace bytes; its contents are scratch and are overwritten).
- * out / lse / softmax_scale / dev_status as for fp_block_sparse_attn. */
+ * fp_sparse_prefill_workspace bytes; its contents are scratch and are overwritten; the work counter
+ * inside it is zeroed by an asynchronous memset on `stream` before the attention launch, and
+ * p->sched is not used). out / lse / softmax_scale / dev_status as for fp_block_sparse_attn. */
 FP_API fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, const void* v, float tau,
                             float softmax_scale, void* workspace, int64_t workspace_bytes, void* out, float* lse,
                             int32_t* dev_status, void* stream);
