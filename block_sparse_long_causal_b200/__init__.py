@@ -6,6 +6,8 @@ CPU or PyTorch fallback: importing this module without the built library raises.
 
 Entry points mirror the C ABI in include/fp.h:
     problem(...)            -> Problem (fp_problem_init)
+    index_buffer_elems(...) -> fp_index_buffer_elems (index buffer length from sequence lengths)
+    check_device_status(..) -> fp_check_device_status (dev_status word -> FpError)
     block_pool(...)         -> fp_block_pool
     block_search(...)       -> fp_block_search
     block_search_topp(...)  -> fp_block_search_topp (the cumulative top-p comparison selector)
@@ -40,7 +42,8 @@ EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_poo
             "fp_dense_attn", "fp_sparse_prefill_workspace", "fp_sparse_prefill", "fp_sparse_prefill_noalloc",
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version", "fp_paged_cache_init",
             "fp_paged_block_pool", "fp_paged_block_search", "fp_paged_block_sparse_attn", "fp_paged_dense_attn",
-            "fp_paged_validate_lists", "fp_block_search_topp", "fp_block_sparse_attn_fp8", "fp_dense_attn_fp8")
+            "fp_paged_validate_lists", "fp_block_search_topp", "fp_block_sparse_attn_fp8", "fp_dense_attn_fp8",
+            "fp_index_buffer_elems", "fp_check_device_status")
 
 
 class FpError(RuntimeError):
@@ -90,6 +93,8 @@ def _load():
         "fp_sparse_prefill_workspace": [P, C.POINTER(C.c_int64)],
         "fp_sparse_prefill": [P, vp, vp, vp, f32, f32, vp, C.c_int64, vp, vp, vp, vp],
         "fp_sparse_prefill_noalloc": [P, vp, vp, vp, f32, f32, vp, vp, vp, vp],
+        "fp_index_buffer_elems": [vp, i32, i32, i32, C.POINTER(C.c_int64)],
+        "fp_check_device_status": [i32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -166,6 +171,21 @@ def problem(cu_seqlens_host, num_q_heads: int, num_kv_heads: int, head_dim: int 
     host = np.ascontiguousarray(cu_seqlens_host, np.int32)
     dev = torch.from_numpy(host.copy()).to(device)
     return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size, work_counter)
+
+
+def index_buffer_elems(seqlens, block_size: int, num_q_heads: int) -> int:
+    """fp_index_buffer_elems: int32 entries of the index buffer for these sequence lengths."""
+    lens = np.ascontiguousarray(seqlens, np.int32)
+    n = C.c_int64(0)
+    _check(_lib.fp_index_buffer_elems(lens.ctypes.data_as(C.c_void_p), len(lens), int(block_size), int(num_q_heads),
+                                      C.byref(n)))
+    return int(n.value)
+
+
+def check_device_status(bits: int) -> None:
+    """fp_check_device_status: raise FpError (status FP_ERR_TIMEOUT / FP_ERR_INVALID_ARG) for a
+    non-zero dev_status word read back after the stream completed."""
+    _check(_lib.fp_check_device_status(int(bits)))
 
 
 def block_pool(p: Problem, q, k, q_pool, k_pool, stream=None):

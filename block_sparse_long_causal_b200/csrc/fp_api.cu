@@ -190,9 +190,78 @@ fp_status set_error(fp_status st, const char* fmt, ...) {
   va_end(ap);
   return st;
 }
+
+unsigned long long context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(a);
+      get_id = reinterpret_cast<GetIdFn>(b);
+    }
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+cudaError_t set_max_smem(const void* func, int bytes, unsigned long long (&done)[kMaxCachedDevices]) {
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kMaxCachedDevices;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached) {
+    const unsigned long long id = context_id();
+    if (id != 0 && done[dev] == id) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) done[dev] = context_id();  // the call above made the context current
+  return e;
+}
 }  // namespace fp
 
 extern "C" {
+
+fp_status fp_index_buffer_elems(const int32_t* host_seqlens, int32_t num_seqs, int32_t block_size,
+                                int32_t num_q_heads, int64_t* out_elems) {
+  if (!host_seqlens || !out_elems) return fail(FP_ERR_INVALID_ARG, "NULL argument to fp_index_buffer_elems");
+  if (num_seqs < 1 || num_seqs > FP_MAX_SEQS)
+    return fail(FP_ERR_INVALID_ARG, "num_seqs=%d outside [1, %d]", num_seqs, FP_MAX_SEQS);
+  if (num_q_heads < 1) return fail(FP_ERR_INVALID_ARG, "num_q_heads=%d must be >= 1", num_q_heads);
+  if (block_size != 64 && block_size != 128)
+    return fail(FP_ERR_UNSUPPORTED, "block_size=%d (64 or 128)", block_size);
+  int64_t idx = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    if (host_seqlens[s] < 0) return fail(FP_ERR_INVALID_ARG, "sequence %d has negative length %d", s, host_seqlens[s]);
+    const int64_t nb = ((int64_t)host_seqlens[s] + block_size - 1) / block_size;
+    idx += (int64_t)num_q_heads * nb * (nb + 1) / 2;
+  }
+  *out_elems = idx;
+  return FP_OK;
+}
+
+fp_status fp_check_device_status(int32_t bits) {
+  if (bits == 0) return FP_OK;
+  const fp_status st = (bits & FP_DEV_TIMEOUT) ? FP_ERR_TIMEOUT : FP_ERR_INVALID_ARG;
+  return fail(st, "device status 0x%x:%s%s%s%s", (unsigned)bits,
+              (bits & FP_DEV_TIMEOUT) ? " a bounded wait gave up (outputs of that launch are undefined);" : "",
+              (bits & FP_DEV_BAD_LIST) ? " an index-list entry or count was out of range (skipped);" : "",
+              (bits & FP_DEV_BAD_PROBLEM) ? " device sequence tables disagreed with the problem (no work done);" : "",
+              (bits & ~(FP_DEV_TIMEOUT | FP_DEV_BAD_LIST | FP_DEV_BAD_PROBLEM)) ? " unknown bits;" : "");
+}
 
 fp_status fp_problem_init(fp_problem* p, const int32_t* host_cu, int32_t num_seqs, const int32_t* dev_cu,
                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size) {
@@ -280,6 +349,7 @@ fp::SearchParams search_params(const fp_problem* p, const fp_paged_cache* c, flo
   a.indices = indices;
   a.index_elems = index_elems(p, c);
   a.dev_status = dev_status;
+  a.wait_limit_ns = wait_limit_ns();
   return a;
 }
 
@@ -532,6 +602,6 @@ fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t
 
 const char* fp_last_error(void) { return g_err; }
 
-int32_t fp_version(void) { return 201; }
+int32_t fp_version(void) { return 300; }
 
 }  // extern "C"

@@ -55,6 +55,7 @@ struct SearchParams {
   int32_t* indices;           // row (s, h, i) at base_s + h*(nb*pb + nb(nb+1)/2) + i*pb + i(i+1)/2
   int64_t index_elems;
   int32_t* dev_status;
+  uint64_t wait_limit_ns;     // limit of every bounded wait of the search kernel
 };
 
 struct ValidateParams {
@@ -93,6 +94,18 @@ constexpr int kTileM = 128;   // query rows per attention tile
 
 // Record the message returned by fp_last_error() and return `st`.
 fp_status set_error(fp_status st, const char* fmt, ...);
+
+// Unique id of the calling thread's current CUDA context (cuCtxGetId), 0 when there is none or the
+// driver cannot tell. Per-device state that a context owns (function attributes, the device address
+// of a static array) is cached under this id, so a context destroyed and created again (for example
+// by cudaDeviceReset) is never mistaken for the old one.
+unsigned long long context_id();
+
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) once per device context: the
+// attribute belongs to the current device's context, so `done[dev]` remembers the context id it was
+// set in (ordinals >= kMaxCachedDevices set it at every call).
+constexpr int kMaxCachedDevices = 64;
+cudaError_t set_max_smem(const void* func, int bytes, unsigned long long (&done)[kMaxCachedDevices]);
 
 cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st);
 cudaError_t launch_search(const SearchParams& p, cudaStream_t st);

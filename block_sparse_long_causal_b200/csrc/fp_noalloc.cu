@@ -14,7 +14,10 @@
 //     it has to start at zero (each call writes every count and list entry before reading it), but
 //     calls that overlap on the GPU (another stream, another host thread) race on it;
 //   - the first call on a device looks up the array's device address (cudaGetSymbolAddress, with that
-//     device current); make that first call before any stream capture;
+//     device current); make that first call before any stream capture. The address is cached per
+//     device under the id of the device's context; a context destroyed and created again (e.g. by
+//     cudaDeviceReset) gets a new id, so the first call after it looks the address up again (make
+//     that call, too, outside stream capture);
 //   - problems whose intermediates exceed FP_NOALLOC_MAX_BYTES are rejected with FP_ERR_INVALID_ARG.
 #include <mutex>
 
@@ -26,11 +29,18 @@ namespace {
 // stand-in, and the kernels receive the address from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FP_NOALLOC_MAX_BYTES];
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = fp::kMaxCachedDevices;
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct CachedAddr {
+  unsigned long long ctx;  // id of the context the address belongs to (0: none cached)
+  void* ptr;
+};
+CachedAddr g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the array on the current device (looked up once per device, then cached).
+// Device address of the array in the current device's context. Looked up once per context with
+// cudaGetSymbolAddress and cached under the context's unique id: after the context is destroyed and
+// created again (cudaDeviceReset), the module is loaded anew, its array may sit elsewhere, and the
+// changed id makes the next call look the address up again.
 fp_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -38,15 +48,17 @@ fp_status scratch_address(void** out) {
     return fp::set_error(FP_ERR_CUDA, "no current CUDA device: %s", cudaGetErrorString(e));
   if (dev >= kMaxDevices) return fp::set_error(FP_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long id = fp::context_id();
+  if (id == 0 || g_scratch_addr[dev].ctx != id || !g_scratch_addr[dev].ptr) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || !ptr)
       return fp::set_error(FP_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s",
                            cudaGetErrorString(e));
-    g_scratch_addr[dev] = ptr;
+    g_scratch_addr[dev].ctx = fp::context_id();  // the lookup made the context current
+    g_scratch_addr[dev].ptr = ptr;
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch_addr[dev].ptr;
   return FP_OK;
 }
 

@@ -61,7 +61,7 @@ typedef enum fp_status {
   FP_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer, non-finite tau, ... */
   FP_ERR_UNSUPPORTED = 2,  /* valid but not implemented here (head_dim != 128, B not 64/128) */
   FP_ERR_CUDA = 3,         /* a CUDA launch or driver call failed */
-  FP_ERR_TIMEOUT = 4       /* reserved for callers that map FP_DEV_TIMEOUT to a status */
+  FP_ERR_TIMEOUT = 4       /* fp_check_device_status: a kernel's bounded wait gave up (FP_DEV_TIMEOUT) */
 } fp_status;
 
 /* Bits written into dev_status by the kernels. */
@@ -95,6 +95,25 @@ typedef struct fp_problem {
  * streams, no ordering between them) must not share them. The results are identical either way.
  * fp_sparse_prefill(_noalloc) use words inside their workspace and ignore sched. */
 #define FP_SCHED_WORDS 2
+
+/* Length, in int32 entries, of the index buffer of a problem: sum_s Hq * nb_s (nb_s + 1) / 2 with
+ * nb_s = ceil(L_s / block_size) (the triangular layout above: query block i of a sequence keeps at
+ * most its i + 1 causal blocks). host_seqlens: HOST array of the num_seqs sequence LENGTHS L_s (not
+ * cumulative offsets), read only during the call. The same value is stored by fp_problem_init in
+ * fp_problem.index_elems; this call gives it to a caller that sizes buffers before it has a device
+ * cu_seqlens. Host-only, nothing is enqueued. FP_ERR_INVALID_ARG for a NULL pointer, num_seqs outside
+ * [1, FP_MAX_SEQS], a negative length or num_q_heads < 1; FP_ERR_UNSUPPORTED for block_size other
+ * than 64 or 128. */
+FP_API fp_status fp_index_buffer_elems(const int32_t* host_seqlens, int32_t num_seqs, int32_t block_size,
+                                       int32_t num_q_heads, int64_t* out_elems);
+
+/* Status of the device work behind a dev_status word that the caller read back after the stream
+ * completed: FP_OK for 0; FP_ERR_TIMEOUT when FP_DEV_TIMEOUT is set (a bounded wait gave up and
+ * that launch's outputs are undefined); otherwise FP_ERR_INVALID_ARG when FP_DEV_BAD_LIST or
+ * FP_DEV_BAD_PROBLEM is set (device-side inputs disagreed with the problem: index entries out of
+ * range, cu_seqlens or prefix lengths that differ from the host copies). fp_last_error() then names
+ * every bit that was set. Host-only, nothing is enqueued. */
+FP_API fp_status fp_check_device_status(int32_t dev_status_bits);
 
 /* Fill *p from a HOST copy of cu_seqlens (read only during the call) and the device copy that the
  * kernels will read. Checks sizes and the sequence limits. */
@@ -269,7 +288,9 @@ FP_API fp_status fp_paged_validate_lists(const fp_problem* p, const fp_paged_cac
  * Every GPU that loads the library holds that array until the process exits. All calls on a device
  * share it and it keeps the last call's contents (nothing needs to start at zero); calls that overlap
  * on the GPU (other streams or threads) race on it. The first call on a device looks up the array's
- * address with that device current: make it before any stream capture. Problems whose intermediates
+ * address with that device current: make it before any stream capture. The address is cached for the
+ * device's current context; after the context is destroyed and created again (cudaDeviceReset), the
+ * next call looks it up again and, like the first, belongs outside stream capture. Problems whose intermediates
  * (fp_sparse_prefill_workspace) exceed FP_NOALLOC_MAX_BYTES return FP_ERR_INVALID_ARG.
  * Arguments as for fp_sparse_prefill, without the workspace. */
 FP_API fp_status fp_sparse_prefill_noalloc(const fp_problem* p, const void* q, const void* k, const void* v,

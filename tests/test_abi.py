@@ -215,3 +215,74 @@ def test_topp_rejects_bad_arguments_before_launch():
                                         None) == fp.FP_ERR_INVALID_ARG
     assert fp._lib.fp_block_search_topp(C.byref(p), ok, ok, C.c_float(0.9), None, ok, ok, None,
                                         None) == fp.FP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("lens,B,hq", [([300], 128, 4), ([300, 1, 400, 0], 64, 3), ([131072], 128, 32),
+                                       ([4096, 8192, 16384, 32768, 65536, 4096, 131072, 2048], 128, 32)])
+def test_index_buffer_elems_is_the_triangular_count(lens, B, hq):
+    nb = [(L + B - 1) // B for L in lens]
+    want = sum(hq * n * (n + 1) // 2 for n in nb)
+    assert fp.index_buffer_elems(lens, B, hq) == want
+    st, p = _prob(tuple(np.concatenate([[0], np.cumsum(lens)]).tolist()), hq=hq, hkv=1, B=B)
+    assert st == fp.FP_OK and p.index_elems == want
+
+
+@pytest.mark.parametrize("lens,B,hq,status", [([], 128, 4, fp.FP_ERR_INVALID_ARG),
+                                              ([5, -1], 128, 4, fp.FP_ERR_INVALID_ARG),
+                                              ([5], 128, 0, fp.FP_ERR_INVALID_ARG),
+                                              ([5], 96, 4, fp.FP_ERR_UNSUPPORTED)])
+def test_index_buffer_elems_rejects(lens, B, hq, status):
+    arr = np.array(lens if lens else [0], np.int32)
+    n = C.c_int64(-7)
+    st = fp._lib.fp_index_buffer_elems(arr.ctypes.data_as(C.c_void_p), len(lens), B, hq, C.byref(n))
+    assert st == status and _err()
+    assert n.value == -7
+    assert fp._lib.fp_index_buffer_elems(None, 1, 128, 4, C.byref(n)) == fp.FP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bits,status,words", [
+    (0, fp.FP_OK, []),
+    (fp.FP_DEV_TIMEOUT, fp.FP_ERR_TIMEOUT, ["bounded wait"]),
+    (fp.FP_DEV_BAD_LIST, fp.FP_ERR_INVALID_ARG, ["out of range"]),
+    (fp.FP_DEV_BAD_PROBLEM, fp.FP_ERR_INVALID_ARG, ["sequence tables"]),
+    (fp.FP_DEV_TIMEOUT | fp.FP_DEV_BAD_LIST, fp.FP_ERR_TIMEOUT, ["bounded wait", "out of range"]),
+])
+def test_check_device_status_maps_the_device_bits(bits, status, words):
+    assert fp._lib.fp_check_device_status(bits) == status
+    if status != fp.FP_OK:
+        msg = _err()
+        assert all(w in msg for w in words), msg
+        with pytest.raises(fp.FpError) as e:
+            fp.check_device_status(bits)
+        assert e.value.status == status
+    else:
+        fp.check_device_status(0)
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """ctypes mirrors of fp_problem and fp_paged_cache have the C sizes and offsets (the header
+    compiled by the host C compiler), and the ABI version is the one of this layout."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = {"fp_problem": [f[0] for f in fp.fp_problem._fields_],
+              "fp_paged_cache": [f[0] for f in fp.fp_paged_cache._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fp.h"', "int main(void) {"]
+    for st, fl in fields.items():
+        lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
+        for f in fl:
+            lines.append(f'  printf("{st} {f} %zu\\n", offsetof({st}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = dict(line.rsplit(" ", 1) for line in subprocess.check_output([str(exe)], text=True).splitlines())
+    for st, cls in (("fp_problem", fp.fp_problem), ("fp_paged_cache", fp.fp_paged_cache)):
+        assert int(got[f"{st} size"]) == C.sizeof(cls)
+        for f in fields[st]:
+            assert int(got[f"{st} {f}"]) == getattr(cls, f).offset, (st, f)
+    assert C.sizeof(fp.fp_problem) == 56 and C.sizeof(fp.fp_paged_cache) == 40
+    assert fp.version() == 300
