@@ -17,20 +17,22 @@
 //   WG1, WG2  softmax of slot 0 / slot 1: thread r owns query row r of its slot's tile (its TMEM
 //                lane): tcgen05.ld of S, causal mask on diagonal tiles, running max in log2 units
 //                (no max pass on unmasked items once the row has one), exp2 on MUFU (an FMA-pipe
-//                polynomial can take a share, kPolyPairs), P packed to bf16 back into the S
-//                columns, lazy O rescale (only when the max grows by more than 2^8), final
-//                normalisation and the bf16 store of O and the LSE.
+//                polynomial share measured slower: it lengthens the softmax's dependency chains more
+//                than it relieves MUFU), P packed to bf16 back into the S columns, lazy O rescale
+//                (only when the max grows by more than 2^8), final normalisation and the bf16 store
+//                of O and the LSE.
 // Registers: setmaxnreg moves WG0 down to 104 and WG1/WG2 up to 200 per thread
 // (128*104 + 256*200 = 384*168, the launch allocation of __launch_bounds__(384, 1)).
 //
-// A work unit pairs two Q tiles that read the same K/V stream, so each K/V tile is loaded once
-// into shared memory for both (GQA packing):
-//   G = Hq/Hkv even: q-heads (2p, 2p+1) of one kv-head, same query tile;
-//   G odd:           one q-head, query tiles (2m+1, 2m) (the last may run alone).
-// The kv iteration is the ascending union of the slots' lists (two per slot when B = 64, where a
-// 128-row tile holds two query blocks); a per-(slot, half) bit masks rows whose list lacks the
-// current block, so different lists stay exact, and a slot none of whose lists holds the block
-// skips the item altogether (no QK, PV or softmax for it).
+// A work unit pairs two Q tiles that read the same K/V stream, so a K/V tile both need is loaded
+// once into shared memory for both (GQA packing): query tiles (2m+1, 2m) of one q-head (the last
+// tile of an odd count runs alone). Each slot walks its own lists (two per slot when B = 64, where a
+// 128-row tile holds two query blocks); a block both slots hold is one item for both, a block of one
+// slot an item of that slot alone (the other skips its QK, PV and softmax), and a per-(slot, half)
+// bit masks rows whose list lacks the item's block, so different lists stay exact. Single-slot
+// items alternate between the slots wherever that loses no shared block, and a slot's QK is issued
+// ahead of the other slot's pending PV, so one slot's softmax overlaps the other's MMAs whether the
+// items are shared or not.
 // Because QK_k(n) is issued after PV_k(n-1) and tcgen05.commit tracks all earlier MMAs, a slot
 // that sees S_k(n) may rescale O_k without waiting: PV_k(n-1) has already completed.
 // Units are ordered kv-head outermost, then by descending query tile, so concurrent CTAs stream
@@ -57,11 +59,6 @@ constexpr int kRegsCtl = 104;       // WG0 (producer, MMA, idle)
 constexpr int kRegsSoftmax = 200;  // WG1, WG2
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax == kThreads * 168,
               "register split must equal the launch allocation");
-// exp2 pairs (index mod 8) evaluated by the FMA-pipe polynomial instead of MUFU. Measured on the
-// 128K causal workload, each poly pair lengthens the softmax's dependency chains more than it
-// relieves MUFU (0 of 8: 187 M cycles per CTA, 2/8: 201 M, 3/8: 205 M, 4/8: 210 M), so every exp2
-// currently goes to MUFU; the split stays for when MUFU throughput becomes the bound.
-constexpr unsigned kPolyPairs = 0x00u;
 // Limit of the waits that only let already-issued copies / MMAs finish on the abort path.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 // Item ring: the producer merges the index lists once and publishes, per unit, the unit's index,
@@ -122,8 +119,12 @@ struct Unit {
   int pb;           // cached prefix blocks: query block i is key block pb + i
 };
 
-// Unit order inside a sequence: kv-head outermost, then descending query tile, then the q-head
-// pairs (G even) or q-heads (G odd) of that kv-head.
+// Unit order inside a sequence: kv-head outermost, then descending query-tile pair, then the
+// q-heads of that kv-head. A unit holds query tiles (2m+1, 2m) of one q-head (the last tile of an odd
+// count runs alone): neighbouring query tiles of a head keep nearly the same key blocks (the sink,
+// the vertical and slash structure repeat from tile to tile), so at sparse settings their lists
+// overlap more than those of two heads at one tile do, and at density 1 they share every block but
+// the upper tile's diagonal.
 __device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s_cb, const int* s_ct,
                                             const int* s_pb, int S, int group) {
   Unit u;
@@ -135,33 +136,20 @@ __device__ __forceinline__ Unit decode_unit(int t, const int* s_cu, const int* s
   u.gb0 = s_cb[u.s];
   u.pb = s_pb[u.s];
   const int ntile = (u.len + kTileM - 1) / kTileM;
-  if ((group & 1) == 0) {
-    const int pairs = group / 2;
-    const int per_g = ntile * pairs;
-    u.g = local / per_g;
-    const int rem = local % per_g;
-    const int qt = ntile - 1 - rem / pairs;
-    const int pr = rem % pairs;
+  const int np = (ntile + 1) / 2;
+  const int per_g = np * group;
+  u.g = local / per_g;
+  const int rem = local % per_g;
+  const int m = np - 1 - rem / group;
+  const int h = u.g * group + rem % group;
+  u.h[0] = u.h[1] = h;
+  if (2 * m + 1 < ntile) {
     u.nslot = 2;
-    u.qt[0] = u.qt[1] = qt;
-    u.h[0] = u.g * group + 2 * pr;
-    u.h[1] = u.h[0] + 1;
+    u.qt[0] = 2 * m + 1;
+    u.qt[1] = 2 * m;
   } else {
-    const int np = (ntile + 1) / 2;
-    const int per_g = np * group;
-    u.g = local / per_g;
-    const int rem = local % per_g;
-    const int m = np - 1 - rem / group;
-    const int h = u.g * group + rem % group;
-    u.h[0] = u.h[1] = h;
-    if (2 * m + 1 < ntile) {
-      u.nslot = 2;
-      u.qt[0] = 2 * m + 1;
-      u.qt[1] = 2 * m;
-    } else {
-      u.nslot = 1;
-      u.qt[0] = u.qt[1] = 2 * m;
-    }
+    u.nslot = 1;
+    u.qt[0] = u.qt[1] = 2 * m;
   }
   return u;
 }
@@ -191,66 +179,131 @@ __device__ __forceinline__ void sched_release(int* sched) {
 }
 
 // ---------------------------------------------------------------------- kv iteration -----------
-// Ascending union of up to four lists: list q = 2*slot + half (half = second query block of a
-// 128-row tile when B = 64). Entries outside [0, own block] are skipped (and reported).
-struct KvIter {
-  const int32_t* l[4];
-  int n[4], i[4], lim[4];
+// One index list of a slot (a 128-row tile holds two query blocks, so two lists, when B = 64).
+// Scalar fields only, so that the walk stays in the producer thread's registers.
+struct ListIter {
+  const int32_t* l;
+  int n, i, lim;
+  int cur;  // valid entry at i (0x7fffffff past the end)
+  int nxt;  // raw entry at i + 1, loaded one step ahead (0x7fffffff past the end)
   bool dense;
+
+  __device__ __forceinline__ int raw(int k) const { return k < n ? (dense ? k : __ldg(l + k)) : 0x7fffffff; }
+  // step to the next valid entry (entries outside [0, lim] are skipped and reported through bad);
+  // the entry after it is loaded now and used at the next step, so the walk waits on no load
+  __device__ __forceinline__ void advance(bool& bad) {
+    ++i;
+    int x = nxt;
+    while (i < n && !(x >= 0 && x <= lim)) {
+      bad = true;
+      ++i;
+      x = raw(i);
+    }
+    cur = i < n ? x : 0x7fffffff;
+    nxt = raw(i + 1);
+  }
+  __device__ __forceinline__ void start(const int32_t* list, int count, int last, bool is_dense, bool& bad) {
+    l = list;
+    n = count;
+    lim = last;
+    dense = is_dense;
+    i = -1;
+    nxt = raw(0);
+    advance(bad);
+  }
+};
+
+// A slot's blocks: the ascending union of its lists.
+struct SlotIter {
+  ListIter a, b;
+
+  __device__ __forceinline__ int first() const { return min(a.cur, b.cur); }
+  // the slot's block after first() (nxt is unchecked: it only steers the order of the two slots)
+  __device__ __forceinline__ int second() const {
+    if (a.cur == b.cur) return min(a.nxt, b.nxt);
+    return a.cur < b.cur ? min(a.nxt, b.cur) : min(b.nxt, a.cur);
+  }
+  // take block j (== first()): the bits of the lists that hold it
+  __device__ __forceinline__ int pop(int j, bool& bad) {
+    int hm = 0;
+    if (a.cur == j) {
+      hm = 1;
+      a.advance(bad);
+    }
+    if (b.cur == j) {
+      hm |= 2;
+      b.advance(bad);
+    }
+    return hm;
+  }
+};
+
+// The unit's item order. A block that both slots' lists hold is one item for both (its K/V tiles
+// are loaded once). A block of one slot only is an item of that slot alone; the MMA issuer then
+// overlaps that slot's softmax with the other slot's MMAs only if the next items alternate between
+// the slots, so when the ascending union would give the same slot two single items in a row, the
+// other slot's next block goes first whenever it is certainly not in the first slot's list (it lies
+// strictly between that list's next two entries), which keeps every shared block shared.
+struct KvIter {
+  SlotIter s0, s1;
+  int last;  // slot (0/1) of the previous single-slot item, -1 after a shared item or at the start
   bool bad;
 
-  __device__ __forceinline__ int peek(int q) {
-    while (i[q] < n[q]) {
-      const int x = dense ? i[q] : __ldg(l[q] + i[q]);
-      if (x >= 0 && x <= lim[q]) return x;
-      bad = true;
-      ++i[q];
-    }
-    return 0x7fffffff;
-  }
   __device__ __forceinline__ bool next(int& j, int& mask) {
-    int v[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = peek(q);
-    j = min(min(v[0], v[1]), min(v[2], v[3]));
-    if (j == 0x7fffffff) return false;
-    mask = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (v[q] == j) {
-        mask |= 1 << q;
-        ++i[q];
-      }
+    const int a = s0.first(), b = s1.first();
+    if (a == 0x7fffffff && b == 0x7fffffff) return false;
+    if (a == b) {
+      j = a;
+      mask = s0.pop(a, bad) | (s1.pop(a, bad) << 2);
+      last = -1;
+      return true;
+    }
+    int pick = a < b ? 0 : 1;
+    if (pick == last && a != 0x7fffffff && b != 0x7fffffff) {
+      if (pick == 0 ? (b < s0.second()) : (a < s1.second())) pick ^= 1;
+    }
+    if (pick == 0) {
+      j = a;
+      mask = s0.pop(a, bad);
+    } else {
+      j = b;
+      mask = s1.pop(b, bad) << 2;
+    }
+    last = pick;
     return true;
   }
 };
 
 template <int BK, bool kCache>
+__device__ __forceinline__ void start_list(ListIter& it, const AttnParams& p, const Unit& u, int k, int hf,
+                                           const int* s_cb, const long long* s_ib, const int* s_pb, bool& bad) {
+  constexpr int per = kTileM / BK;  // query blocks per tile
+  const int blk = u.qt[k] * per + hf;
+  const bool exists = k < u.nslot && hf < per && blk < u.nb;
+  const int jd = (kCache ? u.pb : 0) + blk;  // the query block's diagonal key block
+  const int32_t* list = nullptr;
+  int n = 0;
+  if (exists) {
+    if (p.dense) {
+      n = jd + 1;
+    } else {
+      list = p.indices + list_row(s_cb, s_ib, s_pb, u.s, u.h[k], blk);
+      n = min(max(__ldg(p.counts + (long long)u.h[k] * p.seq.total_blocks + u.gb0 + blk), 0), jd + 1);
+    }
+  }
+  it.start(list, n, jd, p.dense != 0, bad);
+}
+
+template <int BK, bool kCache>
 __device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, const int* s_cb,
                                             const long long* s_ib, const int* s_pb) {
   KvIter it;
+  it.last = -1;
   it.bad = false;
-  it.dense = p.dense != 0;
-  constexpr int per = kTileM / BK;  // query blocks per tile
-  const int NB = p.seq.total_blocks;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int k = q >> 1, hf = q & 1;
-    const int blk = u.qt[k] * per + hf;
-    const bool exists = k < u.nslot && hf < per && blk < u.nb;
-    const int jd = (kCache ? u.pb : 0) + blk;  // the query block's diagonal key block
-    it.i[q] = 0;
-    it.lim[q] = jd;
-    it.l[q] = nullptr;
-    it.n[q] = 0;
-    if (!exists) continue;
-    if (it.dense) {
-      it.n[q] = jd + 1;
-    } else {
-      it.l[q] = p.indices + list_row(s_cb, s_ib, s_pb, u.s, u.h[k], blk);
-      it.n[q] = min(max(__ldg(p.counts + (long long)u.h[k] * NB + u.gb0 + blk), 0), jd + 1);
-    }
-  }
+  start_list<BK, kCache>(it.s0.a, p, u, 0, 0, s_cb, s_ib, s_pb, it.bad);
+  start_list<BK, kCache>(it.s0.b, p, u, 0, 1, s_cb, s_ib, s_pb, it.bad);
+  start_list<BK, kCache>(it.s1.a, p, u, 1, 0, s_cb, s_ib, s_pb, it.bad);
+  start_list<BK, kCache>(it.s1.b, p, u, 1, 1, s_cb, s_ib, s_pb, it.bad);
   return it;
 }
 
@@ -291,7 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
-  const bool even_g = (p.group & 1) == 0;
 
   if (threadIdx.x == 0) {
     mbar_init(b_q_full, 1);
@@ -325,9 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
   }
-  // unit table: G even -> Hq/2 units per 128 query rows; G odd -> Hq units per 256 query rows
-  const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, even_g ? kTileM : 2 * kTileM,
-                                   even_g ? p.hq / 2 : p.hq, s_ok, p.dev_status, s_pb, s_ckb) &&
+  // unit table: Hq units (one per q-head) per 256 query rows (a pair of query tiles)
+  const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, 2 * kTileM, p.hq, s_ok, p.dev_status,
+                                   s_pb, s_ckb) &&
                   (p.dense || s_ib[S] == p.index_elems);
   tc_fence_before();
   __syncthreads();
@@ -372,6 +424,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         ++q_issued;
         KvIter itr = make_iter<BK, kCache>(p, u, s_cb, s_ib, s_pb);
+        // V tile of an item: needed only by its PV, issued after the slot's softmax; it is loaded
+        // after the NEXT item's K tile, so that a V slot still held by a pending PV never delays
+        // the K loads, which the QK MMAs wait for
+        auto load_v = [&](long long vy) -> bool {
+          const int vs = vit % C::kStages;
+          if (!mbar_wait(b_v_empty(vs), ((vit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) return false;
+          mbar_arrive_expect_tx(b_v_full(vs), C::kVBytes);
+          tma_load_2d(sV + vs * C::kVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, (int32_t)vy);
+          tma_load_2d(sV + vs * C::kVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, (int32_t)vy);
+          ++vit;
+          return true;
+        };
+        long long vy = -1;  // V row of the previous item, not loaded yet
         int j, mask;
         while (true) {
           bool more = itr.next(j, mask);
@@ -391,14 +456,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if constexpr (!kFp8)
             tma_load_2d(sK + ks * C::kKBytes + C::kSlabK, &p.tm_k, b_k_full(ks), u.g * kHeadDim + 64, (int32_t)y);
           ++kit;
-          const int vs = vit % C::kStages;
-          if (!mbar_wait(b_v_empty(vs), ((vit / C::kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
-          mbar_arrive_expect_tx(b_v_full(vs), C::kVBytes);
-          tma_load_2d(sV + vs * C::kVBytes, &p.tm_v, b_v_full(vs), u.g * kHeadDim, (int32_t)y);
-          tma_load_2d(sV + vs * C::kVBytes + C::kSlabKV, &p.tm_v, b_v_full(vs), u.g * kHeadDim + 64, (int32_t)y);
-          ++vit;
+          if (vy >= 0 && !load_v(vy)) { fail = true; break; }
+          vy = y;
           if (*s_abort) { fail = true; break; }
         }
+        if (!fail && vy >= 0 && !load_v(vy)) fail = true;  // the unit's last V tile
         bad_list |= itr.bad;
         if (!fail) t = next_unit(p.sched, ++k);
       }
@@ -492,13 +554,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if (!mbar_wait(b_k_full(ks), (kit / C::kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
           const uint32_t kbase = sK + ks * C::kKBytes;
-#pragma unroll
-          for (int sl = 0; sl < 2; ++sl) {
-            if ((prev_part >> sl) & 1) {
-              if (!pv(sl, !had_pv[sl])) { fail = true; break; }
-              had_pv[sl] = true;
+          // A slot that had no part in the previous item issued its last PV earlier: its QK goes
+          // first, so that it does not wait for the other slot's softmax (single-slot items of
+          // alternating slots then overlap like shared ones). A slot that took part issues the
+          // previous item's PV before this item's QK (S_k(n) overwrites P_k(n-1)).
+if (part == 3 && prev_part == 3) {
+            // both slots in both items (every item at density 1): the pingpong order PV0 QK0 PV1 QK1
+            if (!pv(0, !had_pv[0])) { fail = true; break; }
+            had_pv[0] = true;
+            qk(0, kbase);
+            if (!pv(1, !had_pv[1])) { fail = true; break; }
+            had_pv[1] = true;
+            qk(1, kbase);
+          } else {
+  #pragma unroll
+            for (int sl = 0; sl < 2; ++sl)
+              if (((part & ~prev_part) >> sl) & 1) qk(sl, kbase);
+  #pragma unroll
+            for (int sl = 0; sl < 2; ++sl) {
+              if ((prev_part >> sl) & 1) {
+                if (!pv(sl, !had_pv[sl])) { fail = true; break; }
+                had_pv[sl] = true;
+                if ((part >> sl) & 1) qk(sl, kbase);
+              }
             }
-            if ((part >> sl) & 1) qk(sl, kbase);
           }
           if (fail) break;
           if (n > 0) {  // the previous item's PVs are issued: release its V tile
@@ -617,14 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             for (int e = 0; e < 32; e += 2) {
               const int pr = 16 * c + e / 2;  // pair index within the item
               const uint64_t x2 = ffma2(f2_bits(cb[c & 1][e], cb[c & 1][e + 1]), scale2, negm2);
-              uint64_t p2;
-              if ((kPolyPairs >> (pr & 7)) & 1) {
-                p2 = exp2_poly2(x2);
-              } else {
-                float x0, x1;
-                f2_split(x2, x0, x1);
-                p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
-              }
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
               acc[pr & 3] = fadd2(acc[pr & 3], p2);
               float p0, p1;
               f2_split(p2, p0, p1);
@@ -709,18 +783,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
               pk[c / 2] = pack_bf16x2(p0, p1);
             }
           } else {
-            // split exp2 between MUFU and the FMA-pipe polynomial so neither unit alone bounds it
 #pragma unroll
             for (int c = 0; c < BK; c += 2) {
               const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
-              uint64_t p2;
-              if ((kPolyPairs >> ((c >> 1) & 7)) & 1) {
-                p2 = exp2_poly2(x2);
-              } else {
-                float x0, x1;
-                f2_split(x2, x0, x1);
-                p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
-              }
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
               sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
               float p0, p1;
               f2_split(p2, p0, p1);
@@ -797,13 +865,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
 template <int BK, bool kCache, bool kFp8>
 static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<BK, kCache, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<BK, kFp8>::kSmemMax);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static unsigned long long attr_done[kMaxCachedDevices] = {};
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(attn_kernel<BK, kCache, kFp8>), Cfg<BK, kFp8>::kSmemMax,
+                               attr_done);
+  if (e != cudaSuccess) return e;
   attn_kernel<BK, kCache, kFp8><<<grid, kThreads, Cfg<BK, kFp8>::smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }

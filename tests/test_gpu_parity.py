@@ -55,6 +55,14 @@ SMALL = [
     ((900, 385), 6, 2, 128, 0.6, 3.0),      # G = 3: units pair query tiles of one head
     ((1000, 129), 3, 1, 64, 0.7, 3.0),      # G = 3 with B = 64 (four lists per unit)
     ((513,), 2, 2, 128, 0.3, 3.0),          # G = 1, odd tile count (last unit runs one slot)
+    # edge cases of the method
+    ((1000,), 4, 2, 128, 1.0, 3.0),         # tau = 1: argmax ties, sink and diagonal only
+    ((700, 300), 4, 2, 128, 5.0, 3.0),      # tau > 1: sink and diagonal only
+    ((700, 129), 4, 2, 64, -1.0, 3.0),      # tau < 0: every causal block
+    ((700, 0, 500), 4, 2, 128, 0.5, 3.0),   # a zero-length sequence inside a packed batch
+    ((0, 400, 0), 4, 1, 64, 0.6, 3.0),      # zero-length sequences at both ends
+    ((1000, 300), 16, 2, 64, 0.7, 3.0),     # G = 8 with B = 64
+    ((2000,), 16, 2, 64, 0.95, 1.0),        # G = 8 with B = 64, sparse threshold
 ]
 
 
