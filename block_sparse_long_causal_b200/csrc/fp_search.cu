@@ -114,50 +114,24 @@ cudaError_t launch_pool(const PoolParams& p, int grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------------- search ----
-// CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows (q-head, block) that
-// all share the pooled keys of kv-head g (GQA). Row r: head offset r % G, block offset r / G.
-// Scores, row max / min, threshold and emission happen in this one kernel; the block-score matrix
-// is never written to memory. Two CTAs fit on an SM.
-// Pooled keys stream through shared memory in chunks of 64 blocks (cp.async, next chunk in flight).
-// Warp w scores key blocks 8w..8w+7 of a chunk (broadcast shared reads) against rows 2l, 2l+1 of
-// lane l (pooled queries transposed in shared memory).
-// Pass 0 (tensor cores): approximate row max / min of the pooled scores with mma.sync bf16 on a
-// two-term split of the fp32 operands (x = hi + lo; q.k ~ qh.kh + qh.kl + ql.kh) and a rigorous
-// per-row error bound eps_i = 2^-14 * |q_i| * max_j |k_j| / sqrt(d) (the dropped terms and the
-// fp32 accumulation are below 2^-15 * sum_d |q_d k_d| <= 2^-15 * |q| |k|). A row is certainly
-// all-kept when (min - max) - 2 eps >= ln(tau); it is then written as 0..i.
-// If any row of the tile is not certain, the tile takes the exact fp32 path:
-// Pass 1: exact row max m_i and row min of s_ij over j <= i (scores stay in registers); if
-// min - max >= ln(tau) every causal block passes (fp32 subtraction is monotonic, so this is the
-// decision the per-block test would take) and the row is written as 0..i.
-// Pass 2: recompute the exact scores, stage them in shared memory, and one warp per 8 rows emits
-// the kept blocks in ascending order with ballot/popc compaction.
+// --------------------------------------------------------------- fp32 pooled-score tiles ----
+// The exact fp32 pooled scores of a tile (used by the top-p comparison selector, which needs every
+// score of a row): CTA tile = (sequence s, kv-head g, TI consecutive query blocks) -> 64 rows
+// (q-head, block) that share the pooled keys of kv-head g; pooled keys stream through shared memory
+// in chunks of 64 blocks (cp.async, next chunk in flight); warp w scores key blocks 8w..8w+7 of a
+// chunk against rows 2l, 2l+1 of lane l (pooled queries transposed in shared memory).
 constexpr int kSearchThreads = 256;
-constexpr int kSearchWarps = kSearchThreads / 32;
 constexpr int kSearchRows = 64;
 constexpr int kKChunk = 64;                  // key blocks per chunk (8 per warp)
 constexpr int kQTStride = kSearchRows + 4;   // transposed pooled-query row stride (floats)
 constexpr int kKStride = kHeadDim + 4;       // pooled-key row stride (floats), 16-byte aligned
 
 // Shared memory: fixed part, then the sequence tables sized for this launch's sequence count.
-// k[1] doubles as the pass-2 score tile (see the assert).
 struct SearchSmem {
   float k[2][kKChunk][kKStride];             // pooled keys, natural layout, two buffers
   float qT[kHeadDim][kQTStride];             // pooled queries, [d][row]
-  float red[2][kSearchWarps][kSearchRows];   // per-warp row max / min
-  float qnorm[kSearchRows];                  // |q_row| (pass 0 error bound)
-  int kmax_bits;                             // max |k_j| of the tile's keys, as float bits
   int ok;
-  int need_pass2;
-  int need_exact;
 };
-// Pass-0 operand views: split bf16 [hi/lo][row][kBfStride] in the qT region (queries) and in the
-// key region (keys); the padded stride keeps the 32-bit fragment loads conflict free.
-constexpr int kBfStride = kHeadDim + 8;
-static_assert(2 * kSearchRows * kBfStride * 2 <= (int)sizeof(float) * kHeadDim * kQTStride, "query split view");
-static_assert(2 * kKChunk * kBfStride * 2 <= (int)sizeof(float) * 2 * kKChunk * kKStride, "key split view");
-static_assert(kSearchRows * (kKChunk + 1) <= kKChunk * kKStride, "score tile must fit in one key buffer");
 
 __host__ __device__ inline size_t search_smem_bytes(int num_seqs) {
   return sizeof(SearchSmem) + (size_t)(num_seqs + 1) * (5 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
@@ -207,131 +181,122 @@ __device__ __forceinline__ void chunk_scores(const SearchSmem& sm, int buf, int 
   }
 }
 
-__device__ __forceinline__ uint32_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+// ---------------------------------------------------------------------------------- search ----
+// CTA tile = (sequence s, kv-head g, TI = 128 / G consecutive query blocks) -> up to 128 rows
+// (query block i, q-head h) that all read the pooled keys of kv-head g (GQA); row r is block
+// i0 + r / G of q-head g*G + r % G and owns TMEM lane r. One persistent CTA per SM, 9 warps:
+//   warps 0-3  rows: thread r splits its pooled query into bf16 hi + lo (q = qh + ql + O(2^-16 q))
+//              and stores both into TMEM; it reads its row of every score chunk from TMEM;
+//   warps 4-7  converters: thread t splits pooled key j0 + t of each 128-key chunk into bf16 hi + lo
+//              128-byte-swizzled K-major tiles in shared memory, and tracks the largest |k|;
+//   warp 8     allocates TMEM and issues the tcgen05 MMAs from one thread:
+//              acc = qh.kh + qh.kl + ql.kh (A from TMEM, B from shared memory, fp32 accumulate),
+//              so acc = qbar . kbar = sqrt(d) * s_ij up to |err| <= eps = 2^-13 |qbar| max_j |kbar_j|
+//              (the dropped products are below 2^-14.4 sum_d |q_d k_d| and the fp32 accumulation of
+//              the 384 products below 2^-17 of it in any order the tensor core may take; both sums
+//              are at most |q| |k|, so eps holds with a factor 2 to spare).
+// Score chunks flow through a two-stage pipeline: while the rows read chunk c from TMEM, the MMAs
+// of chunk c+1 run and the converters fill the shared buffer of chunk c+2.
+// Pass A: per row, max and min of acc over the row's causal keys (j <= i). The threshold test
+// s_ij - max_j s_ij >= ln(tau) reads acc_j >= max acc + sqrt(d) ln(tau) in these units, and
+// |(acc_j - max acc) - sqrt(d) (s_ij - max_j s_ij)| <= 2 eps. A row with (min - max) - 2 eps >=
+// sqrt(d) ln(tau) keeps every causal block for certain; a tile whose rows all do is written as
+// 0..i and skips pass B.
+// Pass B: recompute the chunks and keep block j iff acc_j >= max acc + sqrt(d) ln(tau) (plus the
+// sink j = 0 and the diagonal). When 2 eps / sqrt(d) <= 0.99e-4 this decision can differ from the
+// exact one only for blocks with |s_ij - max_j s_ij - ln(tau)| < 2 eps / sqrt(d), i.e. inside the
+// tie band |p_ij / max p - tau| <= 1e-4 tau, where either decision is correct (the method's own
+// tolerance); the rows obey it exactly everywhere else. Kept blocks become per-row keep masks,
+// emitted in ascending order by the row's warp with coalesced stores.
+// A row whose bound is wider than that (pooled vectors of very large norm; none in the synthetic
+// workloads) takes an exact fp32 pass instead: its warp computes every score in fp32, the row max,
+// and writes the list in place.
+constexpr int kSrchThreads = 288;
+constexpr int kSrchRows = 128;                      // rows per tile = TMEM lanes
+constexpr int kSrchKeys = 128;                      // pooled keys per chunk = MMA N = TMEM columns per score buffer
+constexpr uint32_t kSrchTmemCols = 512;             // S0 | S1 | Qhi | Qlo (384 columns used)
+constexpr uint32_t kTmS0 = 0, kTmQh = 256, kTmQl = 320;
+constexpr uint32_t kKSlab = kSrchKeys * 128;        // one 64-dim slab of a bf16 key tile (128-byte rows)
+constexpr uint32_t kKTile = 2 * kKSlab;             // bf16 key tile (128 dims)
+constexpr uint32_t kKBuf = 2 * kKTile;              // hi tile | lo tile
+constexpr float kEpsFactor = 1.0f / 8192.0f;        // 2^-13
+constexpr float kBandHalf = 0.99e-4f;               // below the tie band's half width in ln units
+constexpr uint32_t kIdescSearch = idesc_bf16_f32(128, kSrchKeys, 0, 0);
 
-// Split 4 fp32 values into bf16 hi and lo (x - hi) and store them at hi_dst / lo_dst (8 bytes each).
-__device__ __forceinline__ void split_store4(uint16_t* hi_dst, uint16_t* lo_dst, float4 v) {
-  const float x[4] = {v.x, v.y, v.z, v.w};
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    h[e] = bf16_bits(x[e]);
-    l[e] = bf16_bits(x[e] - __uint_as_float(h[e] << 16));
-  }
-  *reinterpret_cast<uint2*>(hi_dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
-  *reinterpret_cast<uint2*>(lo_dst) = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+struct SrchSmem {                  // placed at a 1024-byte aligned address
+  unsigned char k[2][kKBuf];       // key chunk buffers
+  uint64_t bar_s[2];               // the MMAs of the chunk in buffer b have completed
+  uint64_t bar_drain;              // every MMA issued so far has completed (before TMEM is freed)
+  uint32_t tmem_base;
+  int kmax2_bits;                  // max |kbar_j|^2 over the tile's keys (float bits; >= 0 so int order)
+  int need_b;                      // some row of the tile needs pass B
+  int need_exact;                  // some row of the tile needs the exact pass
+  int ok;
+};
+
+__host__ __device__ inline size_t srch_smem_bytes(int num_seqs) {
+  return sizeof(SrchSmem) + 1024 + (size_t)(num_seqs + 1) * (5 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
 }
 
-// 64 rows x 128 fp32 (rows via row_ptr) -> split bf16 view; optional per-row norms.
-// Warp w handles rows w, w + 8, ...; lane l the 4 columns 4l..4l+3.
-template <typename RowPtr>
-__device__ __forceinline__ void load_split_rows(uint16_t* view, RowPtr row_ptr, float* norms, int* max_bits) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kPer = kSearchRows / kSearchWarps;
-  float4 vv[kPer];  // all loads in flight before any use (L2 latency paid once)
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const float* src = row_ptr(warp + q * kSearchWarps);
-    vv[q] = src ? reinterpret_cast<const float4*>(src)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int r = warp + q * kSearchWarps;
-    const float4 v = vv[q];
-    split_store4(view + r * kBfStride + 4 * lane, view + (kSearchRows + r) * kBfStride + 4 * lane, v);
-    float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) {
-      const float nrm = sqrtf(ss);
-      if (norms) norms[r] = nrm;
-      if (max_bits) atomicMax(max_bits, __float_as_int(nrm));
-    }
-  }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Pass-0 key staging: fp32 chunk [64 rows][128] (unpadded) in the upper half of the key region, filled
-// by cp.async while the previous chunk's MMAs run.
-constexpr int kStageOffBytes = 2 * kKChunk * kBfStride * 2;
-static_assert(kStageOffBytes + kKChunk * kHeadDim * 4 <= (int)sizeof(float) * 2 * kKChunk * kKStride, "staging");
-
-__device__ __forceinline__ void issue_stage_chunk(float* stage, const float* kp, int gb0, int g, int hkv, int j0,
-                                                  int jmax) {
-  for (int e = threadIdx.x; e < kKChunk * (kHeadDim / 4); e += kSearchThreads) {
-    const int jr = e / (kHeadDim / 4), c4 = e % (kHeadDim / 4);
-    const int j = min(j0 + jr, jmax);
-    cp_async16(stage + jr * kHeadDim + 4 * c4, kp + ((long long)(gb0 + j) * hkv + g) * kHeadDim + 4 * c4,
-               j0 + jr <= jmax);
+// Exact fp32 dot product of two pooled rows (fixed summation order).
+__device__ __forceinline__ float dot128(const float* a, const float* b) {
+  float s = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < kHeadDim; d += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(a + d);
+    const float4 y = *reinterpret_cast<const float4*>(b + d);
+    s = fmaf(x.x, y.x, s);
+    s = fmaf(x.y, y.y, s);
+    s = fmaf(x.z, y.z, s);
+    s = fmaf(x.w, y.w, s);
   }
-  cp_async_commit();
+  return s;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Pass-0 scores of one 64-block chunk: warp w covers rows 16(w%4).. and key blocks 32(w/4)..;
-// acc[nt][e]: rows r0+g (e = 0,1) and r0+g+8 (e = 2,3), key blocks n0+8nt+2t+(e&1).
-__device__ __forceinline__ void chunk_scores_tc(const uint16_t* qv, const uint16_t* kv, int warp, int lane,
-                                                float (&acc)[4][4]) {
-  const int g = lane >> 2, t = lane & 3;
-  const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-  auto w32 = [](const uint16_t* base, int row, int col) {
-    return *reinterpret_cast<const uint32_t*>(base + row * kBfStride + col);
-  };
-  const uint16_t* qh = qv;
-  const uint16_t* ql = qv + kSearchRows * kBfStride;
-  const uint16_t* kh = kv;
-  const uint16_t* kl = kv + kKChunk * kBfStride;
-#pragma unroll 2
-  for (int kk = 0; kk < kHeadDim; kk += 16) {
-    const int c0 = kk + 2 * t;
-    const uint32_t ah[4] = {w32(qh, r0 + g, c0), w32(qh, r0 + g + 8, c0), w32(qh, r0 + g, c0 + 8), w32(qh, r0 + g + 8, c0 + 8)};
-    const uint32_t al[4] = {w32(ql, r0 + g, c0), w32(ql, r0 + g + 8, c0), w32(ql, r0 + g, c0 + 8), w32(ql, r0 + g + 8, c0 + 8)};
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int n = n0 + 8 * nt + g;
-      const uint32_t bh0 = w32(kh, n, c0), bh1 = w32(kh, n, c0 + 8);
-      const uint32_t bl0 = w32(kl, n, c0), bl1 = w32(kl, n, c0 + 8);
-      mma_bf16_16816(acc[nt], ah, bh0, bh1);
-      mma_bf16_16816(acc[nt], ah, bl0, bl1);
-      mma_bf16_16816(acc[nt], al, bh0, bh1);
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchParams p) {
-  extern __shared__ __align__(16) unsigned char search_smem_raw[];
-  SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
+__global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchParams p) {
+  extern __shared__ __align__(1024) unsigned char srch_raw[];
+  SrchSmem& sm = *reinterpret_cast<SrchSmem*>(((uintptr_t)srch_raw + 1023) & ~(uintptr_t)1023);
   const int S = p.seq.num_seqs;
-  int* t_cu = reinterpret_cast<int*>(search_smem_raw + sizeof(SearchSmem));
+  int* t_cu = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(&sm) + sizeof(SrchSmem));
   int* t_cb = t_cu + (S + 1);
   int* t_ct = t_cb + (S + 1);
   int* t_pb = t_ct + (S + 1);
   int* t_ckb = t_pb + (S + 1);
   long long* t_ib = reinterpret_cast<long long*>(((uintptr_t)(t_ckb + (S + 1)) + 7) & ~(uintptr_t)7);
-  if (!build_seq_tables(p.seq, t_cu, t_cb, t_ct, t_ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
-                        p.dev_status, t_pb, t_ckb))
-    return;
-  if (t_ib[S] != p.index_elems) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
-    return;
-  }
-  const int G = p.group, TI = p.rows_blocks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NB = p.seq.total_blocks;
-  const unsigned lt_mask = (1u << lane) - 1u;
+  const bool is_row = warp < 4, is_conv = warp >= 4 && warp < 8, is_mma = warp == 8;
 
-  const int num_tiles = t_ct[S];
-  // boustrophedon over the grid: tiles are heaviest first, so alternating direction per round
-  // balances the per-CTA work without a work queue
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.bar_s[0]), 1);
+    mbar_init(smem_u32(&sm.bar_s[1]), 1);
+    mbar_init(smem_u32(&sm.bar_drain), 1);
+    fence_mbar_init();
+  }
+  if (is_mma) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kSrchTmemCols);
+    tmem_relinquish();
+  }
+  const bool ok = build_seq_tables(p.seq, t_cu, t_cb, t_ct, t_ib, p.hq, p.rows_blocks * p.seq.block, p.hkv, &sm.ok,
+                                   p.dev_status, t_pb, t_ckb) &&
+                  t_ib[S] == p.index_elems;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (!ok && blockIdx.x == 0 && threadIdx.x == 0) dev_flag(p.dev_status, kDevBadProblem);
+  const int num_tiles = ok ? t_ct[S] : 0;
+
+  const int G = p.group, TI = p.rows_blocks, NB = p.seq.total_blocks;
+  const float sqrt_d = 1.0f / p.inv_sqrt_d;
+  const float c_tau = p.log_tau * sqrt_d;            // ln(tau) in acc units (-inf: keep all)
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint32_t uses0 = 0u, uses1 = 0u;                   // commits into bar_s[0] / bar_s[1] waited on so far
+
   for (int kr = 0;; ++kr) {
     const int tile = kr * gridDim.x + ((kr & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
     if (tile >= num_tiles) break;
@@ -346,244 +311,304 @@ __global__ void __launch_bounds__(kSearchThreads, 2) search_kernel(const SearchP
     const int gb0 = t_cb[s];   // global query block of local block 0 (pooled queries, counts)
     const int pb = t_pb[s];    // cached prefix blocks: query block i is key block pb + i
     const int kb0 = t_ckb[s];  // global key block of the sequence's key block 0 (pooled keys)
-    const int jmax = pb + i_last;  // last key block any row of the tile attends
-    const int nchunks = jmax / kKChunk + 1;
+    const int jmax = pb + i_last;
+    const int nch = jmax / kSrchKeys + 1;
 
-    __syncthreads();  // previous tile done with shared memory
-    const float* q_src = p.q_pool;  // pooled queries of the tile (global, L2 resident)
-    auto q_row = [&](int r) -> const float* {
-      const int i = i0 + r / G;
-      return (r < TI * G && i <= i_last) ? q_src + ((long long)(gb0 + i) * p.hq + g * G + r % G) * kHeadDim : nullptr;
-    };
+    // ---- this thread's row (rows warps): query block, head, diagonal key block, list start
+    const int r = threadIdx.x;
+    const bool rvalid = is_row && r < TI * G && i0 + r / G <= i_last;
+    const int ri = i0 + r / G, rh = g * G + r % G, rjd = pb + ri;
+    const long long rbase = rvalid ? list_row(t_cb, t_ib, t_pb, s, rh, ri) : 0;
+    const float* qrow = p.q_pool + ((long long)(gb0 + ri) * p.hq + rh) * kHeadDim;
+    float qn2 = 0.f;
     if (threadIdx.x == 0) {
-      sm.need_pass2 = 0;
+      sm.kmax2_bits = 0;
+      sm.need_b = 0;
       sm.need_exact = 0;
-      sm.kmax_bits = 0;
     }
-
-    // emission rows: warp w emits rows 8w..8w+7; row_i is the local query block, row_j the last
-    // key block of the row (its diagonal, pb + i), -1 for padding rows
-    int row_i[8], row_j[8], row_h[8];
+    if (is_row && !p.keep_all) {
+      // split the pooled query into bf16 hi + lo and store both into TMEM (A operand of the MMAs)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int rr = warp * 8 + r;
-      row_i[r] = (rr < TI * G && i0 + rr / G <= i_last) ? i0 + rr / G : -1;
-      row_j[r] = row_i[r] >= 0 ? pb + row_i[r] : -1;
-      row_h[r] = g * G + rr % G;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t wh[32], wl[32];
+#pragma unroll
+        for (int f = 0; f < 16; ++f) {
+          const float4 v = rvalid ? *reinterpret_cast<const float4*>(qrow + 64 * half + 4 * f)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          qn2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, qn2))));
+          const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+          wh[2 * f] = h01;
+          wh[2 * f + 1] = h23;
+          wl[2 * f] = pack_bf16x2(v.x - __uint_as_float(h01 << 16), v.y - __uint_as_float(h01 & 0xffff0000u));
+          wl[2 * f + 1] = pack_bf16x2(v.z - __uint_as_float(h23 << 16), v.w - __uint_as_float(h23 & 0xffff0000u));
+        }
+        tmem_st32(tmem + lane_off + kTmQh + 32 * half, wh);
+        tmem_st32(tmem + lane_off + kTmQl + 32 * half, wl);
+      }
+      tmem_wait_st();
+      tc_fence_before();
     }
-    bool all_keep[8];
-    float rmx[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) { all_keep[r] = true; rmx[r] = 0.f; }
+    float mx = -INFINITY, mn = INFINITY;  // pass A: max / min of acc over the row's causal keys
+    float kmax2 = 0.f;                    // converters: largest |kbar|^2 seen
 
-    if (!p.keep_all) {
-      // ---- pass 0: approximate max / min on tensor cores, with a rigorous error bound
-      uint16_t* qv = reinterpret_cast<uint16_t*>(&sm.qT[0][0]);
-      uint16_t* kvw = reinterpret_cast<uint16_t*>(&sm.k[0][0][0]);
-      __syncthreads();
-      load_split_rows(qv, q_row, sm.qnorm, nullptr);
-      const int g4 = lane >> 2, t4 = lane & 3;
-      const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-      int ri[2];
+    // converter: split pooled key j0 + t of chunk cc into buffer b
+    auto convert = [&](int cc, int b) {
+      const int t = threadIdx.x - 128;
+      const int j = cc * kSrchKeys + t;
+      const bool valid = j <= jmax;
+      const float* src = p.k_pool + ((long long)(kb0 + (valid ? j : 0)) * p.hkv + g) * kHeadDim;
+      unsigned char* hi = sm.k[b];
+      unsigned char* lo = sm.k[b] + kKTile;
+      float n2 = 0.f;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int r = r0 + g4 + 8 * h2;
-        ri[h2] = (r < TI * G && i0 + r / G <= i_last) ? pb + i0 + r / G : -1;
-      }
-      float am[2] = {-INFINITY, -INFINITY}, an[2] = {INFINITY, INFINITY};
-      float* stage = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(kvw) + kStageOffBytes);
-      issue_stage_chunk(stage, p.k_pool, kb0, g, p.hkv, 0, jmax);
-      for (int j0 = 0; j0 <= jmax; j0 += kKChunk) {
-        cp_async_wait_all();
-        __syncthreads();  // staged chunk visible; previous chunk's MMAs done with the split view
-        load_split_rows(kvw, [&](int jr) -> const float* { return stage + jr * kHeadDim; }, nullptr,
-                        &sm.kmax_bits);
-        __syncthreads();  // split view ready; staging free
-        if (j0 + kKChunk <= jmax) issue_stage_chunk(stage, p.k_pool, kb0, g, p.hkv, j0 + kKChunk, jmax);
-        float acc[4][4];
-        chunk_scores_tc(qv, kvw, warp, lane, acc);
+      for (int half = 0; half < 2; ++half) {
+        float4 v[16];
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int f = 0; f < 16; ++f)
+          v[f] = valid ? __ldg(reinterpret_cast<const float4*>(src + 64 * half + 4 * f)) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = j0 + n0 + 8 * nt + 2 * t4 + (e & 1);
-            const int h2 = e >> 1;
-            if (j <= ri[h2]) {
-              const float sc = acc[nt][e] * p.inv_sqrt_d;
-              am[h2] = fmaxf(am[h2], sc);
-              an[h2] = fminf(an[h2], sc);
-            }
-          }
-      }
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-          am[h2] = fmaxf(am[h2], __shfl_xor_sync(0xffffffffu, am[h2], o));
-          an[h2] = fminf(an[h2], __shfl_xor_sync(0xffffffffu, an[h2], o));
-        }
-        if (t4 == 0) {
-          sm.red[0][warp >> 2][r0 + g4 + 8 * h2] = am[h2];
-          sm.red[1][warp >> 2][r0 + g4 + 8 * h2] = an[h2];
+        for (int f = 0; f < 16; ++f) {
+          n2 = fmaf(v[f].x, v[f].x, fmaf(v[f].y, v[f].y, fmaf(v[f].z, v[f].z, fmaf(v[f].w, v[f].w, n2))));
+          const uint32_t h01 = pack_bf16x2(v[f].x, v[f].y), h23 = pack_bf16x2(v[f].z, v[f].w);
+          const uint32_t l01 = pack_bf16x2(v[f].x - __uint_as_float(h01 << 16), v[f].y - __uint_as_float(h01 & 0xffff0000u));
+          const uint32_t l23 = pack_bf16x2(v[f].z - __uint_as_float(h23 << 16), v[f].w - __uint_as_float(h23 & 0xffff0000u));
+          // 128-byte swizzle: 16-byte chunk f/2 of row t sits at chunk (f/2) ^ (t % 8)
+          const uint32_t off = half * kKSlab + t * 128 + ((((uint32_t)f >> 1) ^ ((uint32_t)t & 7u)) << 4) + ((f & 1) << 3);
+          *reinterpret_cast<uint2*>(hi + off) = make_uint2(h01, h23);
+          *reinterpret_cast<uint2*>(lo + off) = make_uint2(l01, l23);
         }
       }
-      __syncthreads();
-      const float kmax = __int_as_float(sm.kmax_bits);
-      bool uncertain = false;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int rr = warp * 8 + r;
-        const float a = fmaxf(sm.red[0][0][rr], sm.red[0][1][rr]);
-        const float b = fminf(sm.red[1][0][rr], sm.red[1][1][rr]);
-        const float eps = 6.103515625e-05f * sm.qnorm[rr] * kmax * p.inv_sqrt_d;  // 2^-14 |q| max|k| / sqrt(d)
-        if (row_i[r] >= 0 && !((b - a) - 2.f * eps >= p.log_tau)) uncertain = true;
+      kmax2 = fmaxf(kmax2, n2);
+    };
+    // MMA thread: acc of chunk in buffer b = qh.kh + qh.kl + ql.kh
+    auto issue = [&](int b) {
+      const uint32_t kh = smem_u32(sm.k[b]), kl = kh + kKTile;
+      const uint32_t d = tmem + kTmS0 + 128u * b;
+#pragma unroll 1
+      for (int part = 0; part < 3; ++part) {
+        const uint32_t a = tmem + (part == 2 ? kTmQl : kTmQh);
+        const uint32_t bb = part == 1 ? kl : kh;
+#pragma unroll 1
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(bb + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024);
+          mma_ts(d, a + 8 * kk, bdesc, kIdescSearch, (part > 0 || kk > 0) ? 1u : 0u);
+        }
       }
-      if (uncertain && lane == 0) atomicOr(&sm.need_exact, 1);
-      __syncthreads();
+      mma_commit(smem_u32(&sm.bar_s[b]));
+    };
+    // rows: wait for the chunk in buffer b and read this row's 128 accumulators
+    auto wait_chunk = [&](int b) -> bool {
+      const bool done = mbar_wait(smem_u32(&sm.bar_s[b]), (b ? uses1 : uses0) & 1u, p.wait_limit_ns);
+      if (b) ++uses1; else ++uses0;
+      return done;
+    };
+    bool fail = false;
 
-      if (sm.need_exact) {
-        // ---- exact fp32 path for this tile
-        for (int e = threadIdx.x; e < kSearchRows * (kHeadDim / 4); e += kSearchThreads) {
-          const int r = e % kSearchRows, d4 = e / kSearchRows;
-          const float* src = q_row(r);
-          const float4 v = src ? reinterpret_cast<const float4*>(src)[d4] : make_float4(0.f, 0.f, 0.f, 0.f);
-          sm.qT[4 * d4 + 0][r] = v.x;
-          sm.qT[4 * d4 + 1][r] = v.y;
-          sm.qT[4 * d4 + 2][r] = v.z;
-          sm.qT[4 * d4 + 3][r] = v.w;
+    // one pass over the tile's key chunks; body(c, b) runs on the rows warps for chunk c (TMEM
+    // score buffer b), after its MMAs completed
+    auto run_pass = [&](auto&& body) {
+      if (is_conv) {
+        convert(0, 0);
+        if (nch > 1) convert(1, 1);
+        fence_proxy_async_smem();
+      }
+      __syncthreads();
+      if (is_mma && lane == 0) {
+        tc_fence_after();
+        issue(0);
+      }
+      for (int c = 0; c < nch; ++c) {
+        const int b = c & 1;
+        if (is_mma && lane == 0 && c + 1 < nch) issue(b ^ 1);
+        if (is_row) {
+          if (!__all_sync(0xffffffffu, wait_chunk(b))) fail = true;
+          tc_fence_after();
+          body(c, tmem + lane_off + kTmS0 + 128u * b);
+          tc_fence_before();
         }
-        issue_k_chunk(sm, 0, p.k_pool, kb0, g, p.hkv, 0, jmax);
-        // scoring rows of this lane (li: the row's last key block)
-        int li[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int r = 2 * lane + e;
-          li[e] = (r < TI * G && i0 + r / G <= i_last) ? pb + i0 + r / G : -1;
-        }
-        float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
-        // ---- pass 1: exact row max / min of the pooled scores
-        for (int c = 0; c < nchunks; ++c) {
-          const int j0 = c * kKChunk;
-          if (c + 1 < nchunks) {
-            __syncthreads();  // buffer (c+1)&1 no longer read
-            issue_k_chunk(sm, (c + 1) & 1, p.k_pool, kb0, g, p.hkv, j0 + kKChunk, jmax);
-            cp_async_wait_all_but_one();
-          } else {
-            cp_async_wait_all();
-          }
-          __syncthreads();
-          float acc[2][8];
-          chunk_scores(sm, c & 1, warp, lane, acc);
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-              if (j0 + 8 * warp + b <= li[e]) {
-                const float sc = acc[e][b] * p.inv_sqrt_d;
-                mx[e] = fmaxf(mx[e], sc);
-                mn[e] = fminf(mn[e], sc);
-              }
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          sm.red[0][warp][2 * lane + e] = mx[e];
-          sm.red[1][warp][2 * lane + e] = mn[e];
+        if (is_conv && c + 2 < nch) {
+          if (!wait_chunk(b)) fail = true;  // the MMAs of chunk c no longer read buffer b
+          convert(c + 2, b);
+          fence_proxy_async_smem();
+        } else if (is_conv) {
+          if (b) ++uses1; else ++uses0;  // keep the phase count in step with the rows
         }
         __syncthreads();
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int rr = warp * 8 + r;
-          float a = -INFINITY, b = INFINITY;
-#pragma unroll
-          for (int w = 0; w < kSearchWarps; ++w) {
-            a = fmaxf(a, sm.red[0][w][rr]);
-            b = fminf(b, sm.red[1][w][rr]);
-          }
-          rmx[r] = a;
-          all_keep[r] = (b - a >= p.log_tau);
-        }
       }
+    };
+
+    if (!p.keep_all) {
+      // ---- pass A: max / min of acc over the causal keys of each row
+      run_pass([&](int c, uint32_t scol) {
+        const int j0 = c * kSrchKeys;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t a[32];
+          tmem_ld32(scol + 32 * q, a);
+          tmem_wait_ld();
+          reg_fence32(a);
+          const int jq = j0 + 32 * q;
+          if (jq + 31 <= rjd) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              mx = fmax3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+              mn = fmin3(mn, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (jq + e <= rjd) {
+                mx = fmaxf(mx, __uint_as_float(a[e]));
+                mn = fminf(mn, __uint_as_float(a[e]));
+              }
+            }
+          }
+        }
+      });
+      if (is_conv) atomicMax(&sm.kmax2_bits, __float_as_int(kmax2));
+      __syncthreads();
     }
-    bool warp_needs = false;
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (row_i[r] >= 0 && !all_keep[r]) warp_needs = true;
-    const int warp_jmax = max(max(max(row_j[0], row_j[1]), max(row_j[2], row_j[3])),
-                              max(max(row_j[4], row_j[5]), max(row_j[6], row_j[7])));
-    if (warp_needs && lane == 0) atomicOr(&sm.need_pass2, 1);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (row_i[r] < 0 || !all_keep[r]) continue;
-      const int i = row_i[r], jl = row_j[r];
-      int32_t* dst = p.indices + list_row(t_cb, t_ib, t_pb, s, row_h[r], i);
-      for (int j = lane; j <= jl; j += 32) dst[j] = j;
-      if (lane == 0) p.counts[(long long)row_h[r] * NB + gb0 + i] = jl + 1;
+    // ---- per-row decision after pass A
+    bool keep_all_row = true, exact_row = false;
+    float thr = 0.f;
+    if (is_row && rvalid && !p.keep_all) {
+      const float eps = kEpsFactor * sqrtf(qn2) * sqrtf(__int_as_float(sm.kmax2_bits));
+      keep_all_row = (mn - mx) - 2.f * eps >= c_tau;
+      exact_row = !keep_all_row && 2.f * eps * p.inv_sqrt_d > kBandHalf;
+      thr = mx + c_tau;
+      if (!keep_all_row && !exact_row) atomicOr(&sm.need_b, 1);
+      if (exact_row) atomicOr(&sm.need_exact, 1);
     }
     __syncthreads();
-    if (!sm.need_pass2) continue;
+    const bool need_b = sm.need_b != 0, need_exact = sm.need_exact != 0;
 
-    // ---- pass 2: recompute the scores and emit kept blocks in ascending order
-    float(*sc)[kKChunk + 1] = reinterpret_cast<float(*)[kKChunk + 1]>(&sm.k[1][0][0]);
-    int cnt[8];
-    int64_t base[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      cnt[r] = 0;
-      base[r] = (row_i[r] >= 0) ? list_row(t_cb, t_ib, t_pb, s, row_h[r], row_i[r]) : 0;
-    }
-    for (int c = 0; c < nchunks; ++c) {
-      const int j0 = c * kKChunk;
-      __syncthreads();
-      issue_k_chunk(sm, 0, p.k_pool, kb0, g, p.hkv, j0, jmax);
-      cp_async_wait_all();
-      __syncthreads();
-      float acc[2][8];
-      chunk_scores(sm, 0, warp, lane, acc);
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) sc[2 * lane + e][8 * warp + b] = acc[e][b] * p.inv_sqrt_d;
-      __syncthreads();
-      if (!warp_needs || j0 > warp_jmax) continue;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        if (row_i[r] < 0 || all_keep[r] || j0 > row_j[r]) continue;
-#pragma unroll
-        for (int h2 = 0; h2 < kKChunk; h2 += 32) {
-          const int j = j0 + h2 + lane;
-          const float v = sc[warp * 8 + r][h2 + lane];
-          const bool keep = j <= row_j[r] && (j == 0 || j == row_j[r] || v - rmx[r] >= p.log_tau);
-          const unsigned bal = __ballot_sync(0xffffffffu, keep);
-          if (keep) p.indices[base[r] + cnt[r] + __popc(bal & lt_mask)] = j;
-          cnt[r] += __popc(bal);
+    if (!need_b) {
+      // ---- every row keeps all of its causal blocks (or needs the exact pass): write 0..i
+      if (is_row) {
+        unsigned todo = __ballot_sync(0xffffffffu, rvalid && keep_all_row);
+        while (todo) {
+          const int rr = __ffs(todo) - 1;
+          todo &= todo - 1;
+          const long long base = __shfl_sync(0xffffffffu, rbase, rr);
+          const int jd = __shfl_sync(0xffffffffu, rjd, rr);
+          for (int j = lane; j <= jd; j += 32) p.indices[base + j] = j;
+          if (lane == rr) p.counts[(long long)rh * NB + gb0 + ri] = jd + 1;
         }
       }
-    }
-    if (lane == 0) {
+    } else {
+      // ---- pass B: keep masks of every chunk, emitted by each row's warp
+      int cnt = 0;  // kept blocks of this thread's row so far
+      const bool emit_row = rvalid && !exact_row;
+      run_pass([&](int c, uint32_t scol) {
+        const int j0 = c * kSrchKeys;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (row_i[r] >= 0 && !all_keep[r]) p.counts[(long long)row_h[r] * NB + gb0 + row_i[r]] = cnt[r];
+        for (int q = 0; q < 4; ++q) {
+          uint32_t a[32];
+          tmem_ld32(scol + 32 * q, a);  // warp-collective: every lane takes part
+          tmem_wait_ld();
+          reg_fence32(a);
+          uint32_t m = 0u;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m |= (__uint_as_float(a[e]) >= thr ? 1u : 0u) << e;
+          w[q] = emit_row ? m : 0u;
+        }
+        if (emit_row) {
+          if (j0 == 0) w[0] |= 1u;  // the sink block
+          if (rjd >= j0 && rjd < j0 + kSrchKeys) w[(rjd - j0) >> 5] |= 1u << ((rjd - j0) & 31);  // the diagonal
+          const int lim = rjd - j0 + 1;  // keys j0 .. j0 + lim - 1 are causal
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int n = lim - 32 * q;
+            if (n <= 0) w[q] = 0u;
+            else if (n < 32) w[q] &= (1u << n) - 1u;
+          }
+        }
+        unsigned live = __ballot_sync(0xffffffffu, (w[0] | w[1] | w[2] | w[3]) != 0u);
+        while (live) {
+          const int rr = __ffs(live) - 1;
+          live &= live - 1;
+          const long long base = __shfl_sync(0xffffffffu, rbase, rr);
+          int n = __shfl_sync(0xffffffffu, cnt, rr);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t word = __shfl_sync(0xffffffffu, w[q], rr);
+            if ((word >> lane) & 1u) p.indices[base + n + __popc(word & lt_mask)] = j0 + 32 * q + lane;
+            n += __popc(word);
+          }
+          if (lane == rr) cnt = n;
+        }
+      });
+      if (emit_row) p.counts[(long long)rh * NB + gb0 + ri] = cnt;
     }
+
+    if (need_exact && is_row) {
+      // ---- exact fp32 pass for rows whose bound is wider than the tie band: the row's warp scores
+      // every causal key in fp32 (the scores go to the row's own list as scratch), takes the max and
+      // compacts the kept blocks in place (writes never pass the entries still to be read)
+      unsigned todo = __ballot_sync(0xffffffffu, rvalid && exact_row);
+      while (todo) {
+        const int rr = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const long long base = __shfl_sync(0xffffffffu, rbase, rr);
+        const int jd = __shfl_sync(0xffffffffu, rjd, rr);
+        const int hh = __shfl_sync(0xffffffffu, rh, rr), ii = __shfl_sync(0xffffffffu, ri, rr);
+        const float* qr = p.q_pool + ((long long)(gb0 + ii) * p.hq + hh) * kHeadDim;
+        float m = -INFINITY;
+        for (int j = lane; j <= jd; j += 32) {
+          const float sc = dot128(qr, p.k_pool + ((long long)(kb0 + j) * p.hkv + g) * kHeadDim) * p.inv_sqrt_d;
+          p.indices[base + j] = __float_as_int(sc);
+          m = fmaxf(m, sc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __syncwarp();
+        int n = 0;
+        for (int jj = 0; jj <= jd; jj += 32) {
+          const int j = jj + lane;
+          const float sc = j <= jd ? __int_as_float(p.indices[base + j]) : -INFINITY;
+          __syncwarp();
+          const bool keep = j <= jd && (j == 0 || j == jd || sc - m >= p.log_tau);
+          const unsigned bal = __ballot_sync(0xffffffffu, keep);
+          if (keep) p.indices[base + n + __popc(bal & lt_mask)] = j;
+          n += __popc(bal);
+          __syncwarp();
+        }
+        if (lane == rr) p.counts[(long long)rh * NB + gb0 + ri] = n;
+      }
+    }
+    if (fail && threadIdx.x == 0) dev_flag(p.dev_status, kDevTimeout);
+    __syncthreads();  // the next tile reuses TMEM, the buffers and the flags
+    if (__syncthreads_or(fail)) break;
   }
+
+  if (is_mma) {
+    // every issued MMA has completed before TMEM is released (own, generous limit: MMAs always finish)
+    if (lane == 0) {
+      mma_commit(smem_u32(&sm.bar_drain));
+      mbar_wait(smem_u32(&sm.bar_drain), 0, 1000000000ull);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (is_mma) tmem_dealloc(tmem, kSrchTmemCols);
 }
 
-cudaError_t launch_search(const SearchParams& p, cudaStream_t st) {
-  static bool attr_done = false;
-  const int smem = (int)search_smem_bytes(p.seq.num_seqs);
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(search_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)search_smem_bytes(kMaxSeqs));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+cudaError_t launch_search(const SearchParams& sp, cudaStream_t st) {
+  static unsigned long long attr_done[kMaxCachedDevices] = {};
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(search_kernel), (int)srch_smem_bytes(kMaxSeqs), attr_done);
+  if (e != cudaSuccess) return e;
+  SearchParams p = sp;
+  p.rows_blocks = kSrchRows / p.group;  // query blocks per tile (G <= 64)
+  const long long tiles = (long long)p.hkv * (p.seq.total_blocks / p.rows_blocks + p.seq.num_seqs);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int cap = 2 * sms;
-  const int grid = p.num_tiles < cap ? p.num_tiles : cap;
+  const int grid = (int)(tiles < sms ? tiles : sms);
   if (grid <= 0) return cudaSuccess;
-  search_kernel<<<grid, kSearchThreads, smem, st>>>(p);
+  search_kernel<<<grid, kSrchThreads, srch_smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }
 
@@ -787,13 +812,10 @@ __global__ void __launch_bounds__(256) topp_select_kernel(const ToppParams p) {
 }
 
 cudaError_t launch_topp(const SearchParams& sp, float gamma, float* scores, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(topp_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)search_smem_bytes(kMaxSeqs));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static unsigned long long attr_done[kMaxCachedDevices] = {};
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topp_score_kernel), (int)search_smem_bytes(kMaxSeqs),
+                               attr_done);
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -801,7 +823,7 @@ cudaError_t launch_topp(const SearchParams& sp, float gamma, float* scores, cuda
   const int grid = sp.num_tiles < cap ? sp.num_tiles : cap;
   if (grid <= 0) return cudaSuccess;
   topp_score_kernel<<<grid, kSearchThreads, (int)search_smem_bytes(sp.seq.num_seqs), st>>>(sp, scores);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ToppParams tp;
   tp.seq = sp.seq;
