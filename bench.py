@@ -253,17 +253,35 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(evs=None):
-        # pool + search in one C-ABI call (pool kernel, then search kernel)
+    def step(evs=None, tau=tau):
+        # pool, search and sparse attention: three C-ABI calls, one kernel each, an event between them
         if evs:
             evs[0].record(stream)
+        fp.block_pool(p, q, k, sp.q_pool, sp.k_pool, stream)
+        if evs:
             evs[1].record(stream)
-        fp.block_pool_search(p, q, k, tau, sp.q_pool, sp.k_pool, sp.counts, sp.indices, sp.dev_status, stream)
+        fp.block_search(p, sp.q_pool, sp.k_pool, tau, sp.counts, sp.indices, sp.dev_status, stream)
         if evs:
             evs[2].record(stream)
         fp.block_sparse_attn(p, q, k, v, sp.counts, sp.indices, 0.0, sp.out, None, sp.dev_status, stream)
         if evs:
             evs[3].record(stream)
+
+    def dense():
+        fp.dense_attn(p, q, k, v, 0.0, sp.out, None, sp.dev_status, stream)
+
+    def interleaved(n, tau):
+        """n (sparse step, dense attention) pairs launched back to back, so that the two kernels of a
+        pair see the same clock and power state. Returns per-pair step and dense times (ms)."""
+        il = [[ev() for _ in range(5)] for _ in range(n)]
+        for e in il:
+            step(e, tau)  # records e[0] .. e[3]
+            dense()
+            e[4].record(stream)
+        torch.cuda.synchronize()
+        return ([e[0].elapsed_time(e[3]) for e in il], [e[3].elapsed_time(e[4]) for e in il],
+                [e[0].elapsed_time(e[1]) for e in il], [e[1].elapsed_time(e[2]) for e in il],
+                [e[2].elapsed_time(e[3]) for e in il])
 
     for _ in range(args.warmup):
         step()
@@ -273,23 +291,16 @@ def run_ours(args):
     # dense baseline (own kernel, same design) for the speedup: interleaved with the sparse step
     # (pool + search, then the sparse attention) launch by launch, so that both see the same clock
     # and power state (a short kernel timed first runs at a higher clock under the power cap)
-    dense_ms = step_il_ms = None
+    dense_ms = step_il_ms = ratio = None
     if not args.no_dense:
         for _ in range(2):
-            fp.dense_attn(p, q, k, v, 0.0, sp.out, None, sp.dev_status, stream)
+            dense()
         torch.cuda.synchronize()
-        nd = max(1, min(3, args.steps))
-        il = [[ev() for _ in range(4)] for _ in range(nd)]
-        for e in il:
-            e[0].record(stream)
-            step()
-            e[1].record(stream)
-            e[2].record(stream)
-            fp.dense_attn(p, q, k, v, 0.0, sp.out, None, sp.dev_status, stream)
-            e[3].record(stream)
-        torch.cuda.synchronize()
-        step_il_ms = sum(e[0].elapsed_time(e[1]) for e in il) / nd
-        dense_ms = sum(e[2].elapsed_time(e[3]) for e in il) / nd
+        st_il, de_il, _, _, _ = interleaved(max(3, args.steps), tau)
+        step_il_ms, dense_ms = float(np.median(st_il)), float(np.median(de_il))
+        r = [d / s_ for d, s_ in zip(de_il, st_il)]
+        ratio = {"median": round(float(np.median(r)), 4), "min": round(min(r), 4), "max": round(max(r), 4),
+                 "pairs": len(r)}
 
     supp = None if args.no_supplementary else supplementary(fp, p, sp, x, q, k, v, tau, stream, w)
 
@@ -322,6 +333,34 @@ def run_ours(args):
     counts = sp.counts[:, : p.total_blocks].cpu().numpy()
     eff_flops, dense_flops = kept_flops(counts, cu, w.block, w.d)
     density = eff_flops / dense_flops
+    pk = peaks()
+
+    # ---- labelled supplementary thresholds (outside the timed step): the same workload at tau values
+    # where the search drops blocks, each step interleaved with the dense kernel for the speedup
+    sparse_settings = []
+    if not args.no_dense and args.sparse_taus:
+        for tau_s in [float(t) for t in args.sparse_taus.split(",")]:
+            for _ in range(2):
+                step(None, tau_s)
+            torch.cuda.synchronize()
+            st_il, de_il, po_il, se_il, at_il = interleaved(max(3, args.sparse_pairs), tau_s)
+            c_s = sp.counts[:, : p.total_blocks].cpu().numpy()
+            eff_s, _ = kept_flops(c_s, cu, w.block, w.d)
+            at_ms = float(np.median(at_il))
+            r = [d / s_ for d, s_ in zip(de_il, st_il)]
+            tf = eff_s / (at_ms * 1e-3) / 1e12
+            sparse_settings.append({
+                "tau": tau_s, "label": "supplementary (workload threshold is %g)" % tau,
+                "density": round(eff_s / dense_flops, 6), "effective_tflop": round(eff_s / 1e12, 4),
+                "step_ms": round(float(np.median(st_il)), 4), "pool_ms": round(float(np.median(po_il)), 4),
+                "search_ms": round(float(np.median(se_il)), 4), "attn_ms": round(at_ms, 4),
+                "dense_ms": round(float(np.median(de_il)), 4), "attn_tflops": round(tf, 2),
+                "attn_frac_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
+                "attn_frac_burst": round(tf / pk["bf16_tflops"], 4),
+                "speedup_vs_own_dense": {"median": round(float(np.median(r)), 4), "min": round(min(r), 4),
+                                         "max": round(max(r), 4), "pairs": len(r)}})
+        step(None, tau)  # leave the workload's own lists in place
+        torch.cuda.synchronize()
 
     # ---- e2e through the C ABI with host buffers (H2D of Q/K/V and D2H of O inside the timed region)
     e2e = None
@@ -368,7 +407,6 @@ def run_ours(args):
     if dense_ms is not None:
         dense_ms, step_il_ms = dense_ms_max, step_il_max
 
-    pk = peaks()
     peak_tf = pk["bf16_tflops_sustained"]
     attn_tflops = eff_flops / (attn_ms * 1e-3) / 1e12
     value = job_flops / (ms_step * 1e-3) / 1e12
@@ -391,19 +429,23 @@ def run_ours(args):
             "seq_len": int(max(w.lens)), "parallelism": f"replicas{ws}",
             "l2": "inputs (Q+K+V %.2f GB) larger than L2; no flush" % (sum(a.nbytes for a in (x['q'], x['k'], x['v'])) / 1e9),
         },
-        "breakdown_ms": {"pool_search": round(search_ms, 4), "sparse_attn": round(attn_ms, 4),
+        "breakdown_ms": {"pool": round(pool_ms, 4), "search": round(search_ms, 4), "sparse_attn": round(attn_ms, 4),
                          "dense_attn": round(dense_ms, 4) if dense_ms else None},
         "sparse_prefill_ms": round(ms_step, 4),
         "effective_tflop": round(eff_flops / 1e12, 4),
         "dense_equiv_tflop": round(dense_flops / 1e12, 4),
         "density": round(density, 6),
-        # dense attention over the sparse step (pool + search + sparse attention), timed interleaved
-        "speedup_vs_own_dense": round(dense_ms / step_il_ms, 4) if dense_ms else None,
+        # dense attention over the sparse step (pool + search + sparse attention), timed interleaved:
+        # the median of the per-pair ratios, with their range
+        "speedup_vs_own_dense": ratio["median"] if ratio else None,
+        "speedup_vs_own_dense_range": ratio,
         "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": round(attn_tflops, 2),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tflops / peak_tf, 4),
                      "peak_source": f"{pk['source']} bf16 sustained",
+                     "peak_burst": pk["bf16_tflops"], "frac_of_burst": round(attn_tflops / pk["bf16_tflops"], 4),
                      "traffic": measured_traffic(f"attn_kernel<{w.block}>", w.name)},
         "search_roofline": None,
+        "sparse_settings": sparse_settings,
         "gpu_launches": 3 * args.steps,
         "supplementary": supp,
         "dev_status": status,
@@ -415,11 +457,22 @@ def run_ours(args):
     search_bytes = (2 * T * (w.hq + w.hkv) * w.d + 2 * 4 * NB * (w.hq + w.hkv) * w.d
                     + 4 * w.hq * NB + 4 * float(counts.sum()))
     s_ms = pool_ms + search_ms
+    # per kernel: pool reads Q and K and writes the pooled tensors; search reads the pooled tensors
+    # and writes the counts and the kept indices
+    pool_bytes = 2 * T * (w.hq + w.hkv) * w.d + 4 * NB * (w.hq + w.hkv) * w.d
+    srch_bytes = 4 * NB * (w.hq + w.hkv) * w.d + 4 * w.hq * NB + 4 * float(counts.sum())
+    gbs = lambda b, ms: round(b / (ms * 1e-3) / 1e9, 1)  # noqa: E731
     line["search_roofline"] = {"bound": "hbm", "kernels": "pool_kernel + search_kernel",
-                               "achieved": round(search_bytes / (s_ms * 1e-3) / 1e9, 1),
+                               "achieved": gbs(search_bytes, s_ms),
                                "peak": pk["hbm_gbs"], "unit": "GB/s",
                                "frac": round(search_bytes / (s_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                               "bytes": search_bytes}
+                               "bytes": search_bytes,
+                               "pool_kernel": {"ms": round(pool_ms, 4), "bytes": pool_bytes,
+                                               "achieved": gbs(pool_bytes, pool_ms),
+                                               "frac": round(gbs(pool_bytes, pool_ms) / pk["hbm_gbs"], 4)},
+                               "search_kernel": {"ms": round(search_ms, 4), "bytes": srch_bytes,
+                                                 "achieved": gbs(srch_bytes, search_ms),
+                                                 "frac": round(gbs(srch_bytes, search_ms) / pk["hbm_gbs"], 4)}}
     if e2e:
         line["e2e"] = {"value": round(job_flops / (e2e["ms"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                        "ms_per_step": round(e2e["ms"], 3), "h2d_bytes_per_step": e2e["h2d"],
@@ -532,6 +585,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-supplementary", action="store_true",
                     help="skip the top-p comparison and FP8 timings reported beside the step")
+    ap.add_argument("--sparse-taus", type=str, default="0.95,0.98",
+                    help="comma-separated supplementary thresholds reported beside the workload's own ('' for none)")
+    ap.add_argument("--sparse-pairs", type=int, default=7,
+                    help="interleaved (sparse step, dense) pairs per supplementary threshold")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
