@@ -60,8 +60,8 @@ SMALL = [
     ((700, 300), 4, 2, 128, 5.0, 3.0),      # tau > 1: sink and diagonal only
     ((700, 129), 4, 2, 64, -1.0, 3.0),      # tau < 0: every causal block
     ((700, 0, 500), 4, 2, 128, 0.5, 3.0),   # a zero-length sequence inside a packed batch
-    ((0, 400, 0), 4, 1, 64, 0.6, 3.0),      # zero-length sequences at both ends
-    ((1000, 300), 16, 2, 64, 0.7, 3.0),     # G = 8 with B = 64
+    ((0, 400, 0), 4, 1, 64, 0.6, 1.0),      # zero-length sequences at both ends
+    ((1000, 300), 16, 2, 64, 0.7, 1.0),     # G = 8 with B = 64
     ((2000,), 16, 2, 64, 0.95, 1.0),        # G = 8 with B = 64, sparse threshold
 ]
 
