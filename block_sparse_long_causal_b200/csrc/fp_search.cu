@@ -225,6 +225,7 @@ constexpr uint32_t kIdescSearch = idesc_bf16_f32(128, kSrchKeys, 0, 0);
 
 struct SrchSmem {                  // placed at a 1024-byte aligned address
   unsigned char k[2][kKBuf];       // key chunk buffers
+  float kstage[kSrchKeys][kHeadDim];  // fp32 pooled keys of the next chunk to convert (cp.async)
   uint64_t bar_s[2];               // the MMAs of the chunk in buffer b have completed
   uint64_t bar_drain;              // every MMA issued so far has completed (before TMEM is freed)
   uint32_t tmem_base;
@@ -232,7 +233,13 @@ struct SrchSmem {                  // placed at a 1024-byte aligned address
   int need_b;                      // some row of the tile needs pass B
   int need_exact;                  // some row of the tile needs the exact pass
   int ok;
+  uint4 mask[kSrchRows];           // pass B: each row's keep masks of the current chunk (4 x 32 keys)
+  long long base[kSrchRows];       // each row's list start
+  int cnt[kSrchRows];              // each row's kept blocks so far
 };
+// Pooled-query staging at the start of a tile (in the key buffers, free then): 128 rows of 132 floats
+constexpr int kQStageStride = kHeadDim + 4;
+static_assert(kSrchRows * kQStageStride * 4 <= 2 * kKBuf, "query staging fits in the key buffers");
 
 __host__ __device__ inline size_t srch_smem_bytes(int num_seqs) {
   return sizeof(SrchSmem) + 1024 + (size_t)(num_seqs + 1) * (5 * sizeof(int)) + 8 + (size_t)(num_seqs + 1) * 8;
@@ -255,6 +262,235 @@ __device__ __forceinline__ float dot128(const float* a, const float* b) {
     s = fmaf(x.w, y.w, s);
   }
   return s;
+}
+
+// Shared-space accesses of the converters (the role functions below are not inlined, so generic
+// pointers would not be known to point at shared memory).
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_u2(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void cp_async16_s(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // 0 source bytes -> 16 zero bytes
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+
+// The role code of the search kernel, one copy each (not inlined): the kernel's 9 warps run three
+// different instruction streams, and a small hot footprint keeps them in the instruction cache.
+
+// Converters: copy this thread's share of the fp32 pooled keys of chunk cc into the staging area:
+// converter warp cw takes keys cw, cw + 4, ..., lane l the 16 bytes at dims 4l..4l+3 of each
+// (coalesced). A thread later converts exactly the bytes it copied.
+__device__ __noinline__ void srch_stage(uint32_t kstage, const float* k_pool, int hkv, int g, int kb0, int jmax,
+                                        int cc) {
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 4;
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) {
+    const int jr = cw + 4 * i;
+    const int j = cc * kSrchKeys + jr;
+    const bool valid = j <= jmax;
+    cp_async16_s(kstage + (jr * kHeadDim + 4 * lane) * 4,
+                 k_pool + ((long long)(kb0 + (valid ? j : 0)) * hkv + g) * kHeadDim + 4 * lane, valid);
+  }
+  cp_async_commit();
+}
+
+// Converters: split the staged chunk into the bf16 hi + lo tiles at kbuf (128-byte swizzle: the
+// 16-byte chunk (l % 16) / 2 of slab row jr sits at chunk ((l % 16) / 2) ^ (jr % 8)). Returns the
+// largest |kbar|^2 among the keys whose total this lane ends up holding.
+__device__ __noinline__ float srch_convert(uint32_t kstage, uint32_t kbuf) {
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 4;
+  const uint32_t slab_off = (lane >> 4) * kKSlab + ((lane & 1) << 3);
+  const uint32_t chunk16 = (lane & 15) >> 1;
+  float kmax2 = 0.f;
+  cp_async_wait_all();
+#pragma unroll 1
+  for (int i0b = 0; i0b < 32; i0b += 8) {
+    float ps[8];  // this lane's share of |kbar|^2 of each of the batch's 8 keys
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t jr = cw + 4 * (i0b + u);
+      const float4 v = lds_f4(kstage + (jr * kHeadDim + 4 * lane) * 4);
+      ps[u] = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
+      const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+      const uint32_t l01 = pack_bf16x2(v.x - __uint_as_float(h01 << 16), v.y - __uint_as_float(h01 & 0xffff0000u));
+      const uint32_t l23 = pack_bf16x2(v.z - __uint_as_float(h23 << 16), v.w - __uint_as_float(h23 & 0xffff0000u));
+      const uint32_t off = slab_off + jr * 128 + ((chunk16 ^ (jr & 7u)) << 4);
+      sts_u2(kbuf + off, h01, h23);
+      sts_u2(kbuf + kKTile + off, l01, l23);
+    }
+    // transpose-reduce over the 32 lanes: three halving exchanges leave each lane one key's partial
+    // sum over 4 lanes, two butterflies finish it
+#pragma unroll
+    for (int sft = 16, nv = 4; sft >= 4; sft >>= 1, nv >>= 1) {
+      const bool upper = (lane & sft) != 0;
+#pragma unroll
+      for (int i = 0; i < nv; ++i) {
+        const float send = upper ? ps[i] : ps[i + nv];
+        const float keep = upper ? ps[i + nv] : ps[i];
+        ps[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+      }
+    }
+    ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], 2);
+    ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], 1);
+    kmax2 = fmaxf(kmax2, ps[0]);
+  }
+  return kmax2;
+}
+
+// MMA thread: acc (TMEM columns d .. d+127) = qh.kh + qh.kl + ql.kh for the key tiles at kbuf.
+__device__ __noinline__ void srch_issue(uint32_t tmem, uint32_t d, uint32_t kbuf, uint32_t bar) {
+  const uint32_t kh = kbuf, kl = kbuf + kKTile;
+#pragma unroll
+  for (int part = 0; part < 3; ++part) {
+    const uint32_t a = tmem + (part == 2 ? kTmQl : kTmQh);
+    const uint32_t bb = part == 1 ? kl : kh;
+#pragma unroll
+    for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+      const uint64_t bdesc = sdesc_sw128(bb + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024);
+      mma_ts(tmem + d, a + 8 * kk, bdesc, kIdescSearch, (part > 0 || kk > 0) ? 1u : 0u);
+    }
+  }
+  mma_commit(bar);
+}
+
+// Rows, pass A: max and min of acc over this row's causal keys of the chunk at TMEM address scol
+// (keys j0 .. j0 + 127; the row's last causal key is jd).
+__device__ __noinline__ float2 srch_pass_a(uint32_t scol, int j0, int jd, float mx, float mn) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a[32];
+    tmem_ld32(scol + 32 * q, a);
+    tmem_wait_ld();
+    reg_fence32(a);
+    const int jq = j0 + 32 * q;
+    if (jq + 31 <= jd) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        mx = fmax3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+        mn = fmin3(mn, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (jq + e <= jd) {
+          mx = fmaxf(mx, __uint_as_float(a[e]));
+          mn = fminf(mn, __uint_as_float(a[e]));
+        }
+    }
+  }
+  return make_float2(mx, mn);
+}
+
+// Rows, pass B: this row's keep mask of the chunk (acc >= thr, the sink, the diagonal, causal keys
+// only), then the warp writes its 32 rows' kept blocks, one row at a time, with coalesced stores.
+// masks / bases / cnts: the tile's per-row arrays in shared memory (shared addresses).
+__device__ __noinline__ void srch_pass_b(uint32_t scol, int j0, int jd, float thr, bool emit, uint32_t masks,
+                                         const long long* bases, int* cnts, int32_t* indices) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a[32];
+    tmem_ld32(scol + 32 * q, a);  // warp-collective: every lane takes part
+    tmem_wait_ld();
+    reg_fence32(a);
+    uint32_t m = 0u;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m |= (__uint_as_float(a[e]) >= thr ? 1u : 0u) << e;
+    w[q] = emit ? m : 0u;
+  }
+  if (emit) {
+    if (j0 == 0) w[0] |= 1u;                                                                // the sink
+    if (jd >= j0 && jd < j0 + kSrchKeys) w[(jd - j0) >> 5] |= 1u << ((jd - j0) & 31);      // the diagonal
+    const int lim = jd - j0 + 1;  // keys j0 .. j0 + lim - 1 are causal
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int n = lim - 32 * q;
+      if (n <= 0) w[q] = 0u;
+      else if (n < 32) w[q] &= (1u << n) - 1u;
+    }
+  }
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(masks + 16u * threadIdx.x), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3])
+               : "memory");
+  __syncwarp();
+#pragma unroll 2
+  for (int rr = 0; rr < 32; ++rr) {
+    const int r2 = 32 * warp + rr;
+    uint4 m;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(m.x), "=r"(m.y), "=r"(m.z), "=r"(m.w) : "r"(masks + 16u * r2));
+    if ((m.x | m.y | m.z | m.w) == 0u) continue;
+    const long long base = bases[r2];
+    int n = cnts[r2];
+    const uint32_t words[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if ((words[q] >> lane) & 1u) indices[base + n + __popc(words[q] & lt_mask)] = j0 + 32 * q + lane;
+      n += __popc(words[q]);
+    }
+    __syncwarp();
+    if (lane == 0) cnts[r2] = n;
+  }
+  __syncwarp();
+}
+
+// Rows of a tile that keeps every causal block: the warp writes 0..jd of each such row of its 32.
+__device__ __noinline__ void srch_write_all(bool mine, long long base, int jd, int32_t* indices, int32_t* count) {
+  const int lane = threadIdx.x & 31;
+  unsigned todo = __ballot_sync(0xffffffffu, mine);
+  while (todo) {
+    const int rr = __ffs(todo) - 1;
+    todo &= todo - 1;
+    const long long b = __shfl_sync(0xffffffffu, base, rr);
+    const int n = __shfl_sync(0xffffffffu, jd, rr) + 1;
+    for (int j = lane; j < n; j += 32) indices[b + j] = j;
+  }
+  if (mine) *count = jd + 1;
+}
+
+// Exact fp32 pass for rows whose bound is wider than the tie band: the row's warp scores every causal
+// key with fp32 FMAs (the scores go to the row's own list as scratch), takes the max and compacts the
+// kept blocks in place (the writes never pass the entries still to be read).
+__device__ __noinline__ void srch_exact_rows(bool mine, long long base, int jd, const float* qrow, const float* k_pool,
+                                             int kb0, int hkv, int g, float inv_sqrt_d, float log_tau,
+                                             int32_t* indices, int32_t* count) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  unsigned todo = __ballot_sync(0xffffffffu, mine);
+  while (todo) {
+    const int rr = __ffs(todo) - 1;
+    todo &= todo - 1;
+    const long long b = __shfl_sync(0xffffffffu, base, rr);
+    const int d = __shfl_sync(0xffffffffu, jd, rr);
+    const float* qr = reinterpret_cast<const float*>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(qrow), rr));
+    float m = -INFINITY;
+    for (int j = lane; j <= d; j += 32) {
+      const float sc = dot128(qr, k_pool + ((long long)(kb0 + j) * hkv + g) * kHeadDim) * inv_sqrt_d;
+      indices[b + j] = __float_as_int(sc);
+      m = fmaxf(m, sc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __syncwarp();
+    int n = 0;
+    for (int jj = 0; jj <= d; jj += 32) {
+      const int j = jj + lane;
+      const float sc = j <= d ? __int_as_float(indices[b + j]) : -INFINITY;
+      __syncwarp();
+      const bool keep = j <= d && (j == 0 || j == d || sc - m >= log_tau);
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if (keep) indices[b + n + __popc(bal & lt_mask)] = j;
+      n += __popc(bal);
+      __syncwarp();
+    }
+    if (lane == rr) *count = n;
+  }
 }
 
 __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchParams p) {
@@ -294,8 +530,12 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
   const float sqrt_d = 1.0f / p.inv_sqrt_d;
   const float c_tau = p.log_tau * sqrt_d;            // ln(tau) in acc units (-inf: keep all)
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  uint32_t uses0 = 0u, uses1 = 0u;                   // commits into bar_s[0] / bar_s[1] waited on so far
+  const uint32_t kstage = smem_u32(&sm.kstage[0][0]);
+  const uint32_t kbuf0 = smem_u32(sm.k[0]), kbuf1 = smem_u32(sm.k[1]);
+  const uint32_t bar0 = smem_u32(&sm.bar_s[0]), bar1 = smem_u32(&sm.bar_s[1]);
+  const uint32_t masks = smem_u32(&sm.mask[0]);
+  uint32_t uses0 = 0u, uses1 = 0u;                   // completions of bar_s[0] / bar_s[1] waited on so far
+  bool fail = false;
 
   for (int kr = 0;; ++kr) {
     const int tile = kr * gridDim.x + ((kr & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
@@ -319,22 +559,38 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
     const bool rvalid = is_row && r < TI * G && i0 + r / G <= i_last;
     const int ri = i0 + r / G, rh = g * G + r % G, rjd = pb + ri;
     const long long rbase = rvalid ? list_row(t_cb, t_ib, t_pb, s, rh, ri) : 0;
-    const float* qrow = p.q_pool + ((long long)(gb0 + ri) * p.hq + rh) * kHeadDim;
+    int32_t* rcount = p.counts + (long long)rh * NB + gb0 + ri;
     float qn2 = 0.f;
     if (threadIdx.x == 0) {
       sm.kmax2_bits = 0;
       sm.need_b = 0;
       sm.need_exact = 0;
     }
+    if (is_row) {
+      sm.base[r] = rbase;
+      sm.cnt[r] = 0;
+    }
     if (is_row && !p.keep_all) {
-      // split the pooled query into bf16 hi + lo and store both into TMEM (A operand of the MMAs)
+      // the pooled queries of this warp's 32 rows: coalesced row copies into the staging area, then
+      // each thread splits its own row into bf16 hi + lo and stores both into TMEM (the A operand of
+      // the MMAs)
+      const uint32_t stage = kbuf0;
+#pragma unroll 8
+      for (int rr = 0; rr < 32; ++rr) {
+        const int r2 = 32 * warp + rr;
+        const bool v2 = r2 < TI * G && i0 + r2 / G <= i_last;
+        const float* src = p.q_pool + ((long long)(gb0 + i0 + (v2 ? r2 / G : 0)) * p.hq + g * G + r2 % G) * kHeadDim;
+        cp_async16_s(stage + (r2 * kQStageStride + 4 * lane) * 4, src + 4 * lane, v2);
+      }
+      cp_async_commit();
+      cp_async_wait_all();
+      __syncwarp();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t wh[32], wl[32];
 #pragma unroll
         for (int f = 0; f < 16; ++f) {
-          const float4 v = rvalid ? *reinterpret_cast<const float4*>(qrow + 64 * half + 4 * f)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 v = lds_f4(stage + (r * kQStageStride + 64 * half + 4 * f) * 4);
           qn2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, qn2))));
           const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
           wh[2 * f] = h01;
@@ -348,239 +604,94 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
       tmem_wait_st();
       tc_fence_before();
     }
+    __syncthreads();  // the staging area becomes the key buffers again
     float mx = -INFINITY, mn = INFINITY;  // pass A: max / min of acc over the row's causal keys
     float kmax2 = 0.f;                    // converters: largest |kbar|^2 seen
+    bool keep_all_row = true, exact_row = false, need_b = false;
+    float thr = 0.f;
 
-    // converter: split pooled key j0 + t of chunk cc into buffer b
-    auto convert = [&](int cc, int b) {
-      const int t = threadIdx.x - 128;
-      const int j = cc * kSrchKeys + t;
-      const bool valid = j <= jmax;
-      const float* src = p.k_pool + ((long long)(kb0 + (valid ? j : 0)) * p.hkv + g) * kHeadDim;
-      unsigned char* hi = sm.k[b];
-      unsigned char* lo = sm.k[b] + kKTile;
-      float n2 = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float4 v[16];
-#pragma unroll
-        for (int f = 0; f < 16; ++f)
-          v[f] = valid ? __ldg(reinterpret_cast<const float4*>(src + 64 * half + 4 * f)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int f = 0; f < 16; ++f) {
-          n2 = fmaf(v[f].x, v[f].x, fmaf(v[f].y, v[f].y, fmaf(v[f].z, v[f].z, fmaf(v[f].w, v[f].w, n2))));
-          const uint32_t h01 = pack_bf16x2(v[f].x, v[f].y), h23 = pack_bf16x2(v[f].z, v[f].w);
-          const uint32_t l01 = pack_bf16x2(v[f].x - __uint_as_float(h01 << 16), v[f].y - __uint_as_float(h01 & 0xffff0000u));
-          const uint32_t l23 = pack_bf16x2(v[f].z - __uint_as_float(h23 << 16), v[f].w - __uint_as_float(h23 & 0xffff0000u));
-          // 128-byte swizzle: 16-byte chunk f/2 of row t sits at chunk (f/2) ^ (t % 8)
-          const uint32_t off = half * kKSlab + t * 128 + ((((uint32_t)f >> 1) ^ ((uint32_t)t & 7u)) << 4) + ((f & 1) << 3);
-          *reinterpret_cast<uint2*>(hi + off) = make_uint2(h01, h23);
-          *reinterpret_cast<uint2*>(lo + off) = make_uint2(l01, l23);
-        }
-      }
-      kmax2 = fmaxf(kmax2, n2);
-    };
-    // MMA thread: acc of chunk in buffer b = qh.kh + qh.kl + ql.kh
-    auto issue = [&](int b) {
-      const uint32_t kh = smem_u32(sm.k[b]), kl = kh + kKTile;
-      const uint32_t d = tmem + kTmS0 + 128u * b;
-#pragma unroll 1
-      for (int part = 0; part < 3; ++part) {
-        const uint32_t a = tmem + (part == 2 ? kTmQl : kTmQh);
-        const uint32_t bb = part == 1 ? kl : kh;
-#pragma unroll 1
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(bb + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024);
-          mma_ts(d, a + 8 * kk, bdesc, kIdescSearch, (part > 0 || kk > 0) ? 1u : 0u);
-        }
-      }
-      mma_commit(smem_u32(&sm.bar_s[b]));
-    };
-    // rows: wait for the chunk in buffer b and read this row's 128 accumulators
-    auto wait_chunk = [&](int b) -> bool {
-      const bool done = mbar_wait(smem_u32(&sm.bar_s[b]), (b ? uses1 : uses0) & 1u, p.wait_limit_ns);
-      if (b) ++uses1; else ++uses0;
-      return done;
-    };
-    bool fail = false;
-
-    // one pass over the tile's key chunks; body(c, b) runs on the rows warps for chunk c (TMEM
-    // score buffer b), after its MMAs completed
-    auto run_pass = [&](auto&& body) {
+    // ---- pass A (0), then pass B (1) when some row needs it: the same chunk pipeline; while the
+    // rows read chunk c from TMEM, the MMAs of chunk c + 1 run and the converters fill chunk c + 2
+    for (int pass = p.keep_all ? 2 : 0; pass < 2; ++pass) {
+      if (pass == 1 && !need_b) break;
       if (is_conv) {
-        convert(0, 0);
-        if (nch > 1) convert(1, 1);
+        srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 0);
+        kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf0));
+        if (nch > 1) {
+          srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 1);
+          kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf1));
+        }
+        if (nch > 2) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 2);  // lands while the first chunks are scored
         fence_proxy_async_smem();
       }
       __syncthreads();
       if (is_mma && lane == 0) {
         tc_fence_after();
-        issue(0);
+        srch_issue(tmem, kTmS0, kbuf0, bar0);
       }
       for (int c = 0; c < nch; ++c) {
         const int b = c & 1;
-        if (is_mma && lane == 0 && c + 1 < nch) issue(b ^ 1);
+        if (is_mma && lane == 0 && c + 1 < nch) srch_issue(tmem, kTmS0 + 128u * (b ^ 1), b ? kbuf0 : kbuf1, b ? bar0 : bar1);
+        if (is_row || is_conv) {
+          const bool rows = is_row;
+          if (rows || c + 2 < nch) {
+            // the MMAs of chunk c are done: its scores are in TMEM and buffer b is free again
+            const bool done = mbar_wait(b ? bar1 : bar0, (b ? uses1 : uses0) & 1u, p.wait_limit_ns);
+            if (rows ? !__all_sync(0xffffffffu, done) : !done) fail = true;
+          }
+          if (b) ++uses1; else ++uses0;
+        }
         if (is_row) {
-          if (!__all_sync(0xffffffffu, wait_chunk(b))) fail = true;
           tc_fence_after();
-          body(c, tmem + lane_off + kTmS0 + 128u * b);
+          const uint32_t scol = tmem + lane_off + kTmS0 + 128u * b;
+          if (pass == 0) {
+            const float2 v = srch_pass_a(scol, c * kSrchKeys, rjd, mx, mn);
+            mx = v.x;
+            mn = v.y;
+          } else {
+            srch_pass_b(scol, c * kSrchKeys, rjd, thr, rvalid && !exact_row, masks, sm.base, sm.cnt, p.indices);
+          }
           tc_fence_before();
         }
         if (is_conv && c + 2 < nch) {
-          if (!wait_chunk(b)) fail = true;  // the MMAs of chunk c no longer read buffer b
-          convert(c + 2, b);
+          kmax2 = fmaxf(kmax2, srch_convert(kstage, b ? kbuf1 : kbuf0));  // chunk c + 2, staged during chunk c + 1
+          if (c + 3 < nch) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, c + 3);
           fence_proxy_async_smem();
-        } else if (is_conv) {
-          if (b) ++uses1; else ++uses0;  // keep the phase count in step with the rows
         }
         __syncthreads();
       }
-    };
-
-    if (!p.keep_all) {
-      // ---- pass A: max / min of acc over the causal keys of each row
-      run_pass([&](int c, uint32_t scol) {
-        const int j0 = c * kSrchKeys;
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t a[32];
-          tmem_ld32(scol + 32 * q, a);
-          tmem_wait_ld();
-          reg_fence32(a);
-          const int jq = j0 + 32 * q;
-          if (jq + 31 <= rjd) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              mx = fmax3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
-              mn = fmin3(mn, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (jq + e <= rjd) {
-                mx = fmaxf(mx, __uint_as_float(a[e]));
-                mn = fminf(mn, __uint_as_float(a[e]));
-              }
-            }
-          }
+      if (pass == 0) {
+        // ---- per-row decision after pass A
+        if (is_conv) atomicMax(&sm.kmax2_bits, __float_as_int(kmax2));
+        __syncthreads();
+        if (is_row && rvalid) {
+          const float eps = kEpsFactor * sqrtf(qn2) * sqrtf(__int_as_float(sm.kmax2_bits));
+          keep_all_row = (mn - mx) - 2.f * eps >= c_tau;
+          exact_row = !keep_all_row && 2.f * eps * p.inv_sqrt_d > kBandHalf;
+          thr = mx + c_tau;
+          if (!keep_all_row && !exact_row) atomicOr(&sm.need_b, 1);
+          if (exact_row) atomicOr(&sm.need_exact, 1);
         }
-      });
-      if (is_conv) atomicMax(&sm.kmax2_bits, __float_as_int(kmax2));
-      __syncthreads();
-    }
-    // ---- per-row decision after pass A
-    bool keep_all_row = true, exact_row = false;
-    float thr = 0.f;
-    if (is_row && rvalid && !p.keep_all) {
-      const float eps = kEpsFactor * sqrtf(qn2) * sqrtf(__int_as_float(sm.kmax2_bits));
-      keep_all_row = (mn - mx) - 2.f * eps >= c_tau;
-      exact_row = !keep_all_row && 2.f * eps * p.inv_sqrt_d > kBandHalf;
-      thr = mx + c_tau;
-      if (!keep_all_row && !exact_row) atomicOr(&sm.need_b, 1);
-      if (exact_row) atomicOr(&sm.need_exact, 1);
-    }
-    __syncthreads();
-    const bool need_b = sm.need_b != 0, need_exact = sm.need_exact != 0;
-
-    if (!need_b) {
-      // ---- every row keeps all of its causal blocks (or needs the exact pass): write 0..i
-      if (is_row) {
-        unsigned todo = __ballot_sync(0xffffffffu, rvalid && keep_all_row);
-        while (todo) {
-          const int rr = __ffs(todo) - 1;
-          todo &= todo - 1;
-          const long long base = __shfl_sync(0xffffffffu, rbase, rr);
-          const int jd = __shfl_sync(0xffffffffu, rjd, rr);
-          for (int j = lane; j <= jd; j += 32) p.indices[base + j] = j;
-          if (lane == rr) p.counts[(long long)rh * NB + gb0 + ri] = jd + 1;
-        }
-      }
-    } else {
-      // ---- pass B: keep masks of every chunk, emitted by each row's warp
-      int cnt = 0;  // kept blocks of this thread's row so far
-      const bool emit_row = rvalid && !exact_row;
-      run_pass([&](int c, uint32_t scol) {
-        const int j0 = c * kSrchKeys;
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t a[32];
-          tmem_ld32(scol + 32 * q, a);  // warp-collective: every lane takes part
-          tmem_wait_ld();
-          reg_fence32(a);
-          uint32_t m = 0u;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) m |= (__uint_as_float(a[e]) >= thr ? 1u : 0u) << e;
-          w[q] = emit_row ? m : 0u;
-        }
-        if (emit_row) {
-          if (j0 == 0) w[0] |= 1u;  // the sink block
-          if (rjd >= j0 && rjd < j0 + kSrchKeys) w[(rjd - j0) >> 5] |= 1u << ((rjd - j0) & 31);  // the diagonal
-          const int lim = rjd - j0 + 1;  // keys j0 .. j0 + lim - 1 are causal
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int n = lim - 32 * q;
-            if (n <= 0) w[q] = 0u;
-            else if (n < 32) w[q] &= (1u << n) - 1u;
-          }
-        }
-        unsigned live = __ballot_sync(0xffffffffu, (w[0] | w[1] | w[2] | w[3]) != 0u);
-        while (live) {
-          const int rr = __ffs(live) - 1;
-          live &= live - 1;
-          const long long base = __shfl_sync(0xffffffffu, rbase, rr);
-          int n = __shfl_sync(0xffffffffu, cnt, rr);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t word = __shfl_sync(0xffffffffu, w[q], rr);
-            if ((word >> lane) & 1u) p.indices[base + n + __popc(word & lt_mask)] = j0 + 32 * q + lane;
-            n += __popc(word);
-          }
-          if (lane == rr) cnt = n;
-        }
-      });
-      if (emit_row) p.counts[(long long)rh * NB + gb0 + ri] = cnt;
-    }
-
-    if (need_exact && is_row) {
-      // ---- exact fp32 pass for rows whose bound is wider than the tie band: the row's warp scores
-      // every causal key in fp32 (the scores go to the row's own list as scratch), takes the max and
-      // compacts the kept blocks in place (writes never pass the entries still to be read)
-      unsigned todo = __ballot_sync(0xffffffffu, rvalid && exact_row);
-      while (todo) {
-        const int rr = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const long long base = __shfl_sync(0xffffffffu, rbase, rr);
-        const int jd = __shfl_sync(0xffffffffu, rjd, rr);
-        const int hh = __shfl_sync(0xffffffffu, rh, rr), ii = __shfl_sync(0xffffffffu, ri, rr);
-        const float* qr = p.q_pool + ((long long)(gb0 + ii) * p.hq + hh) * kHeadDim;
-        float m = -INFINITY;
-        for (int j = lane; j <= jd; j += 32) {
-          const float sc = dot128(qr, p.k_pool + ((long long)(kb0 + j) * p.hkv + g) * kHeadDim) * p.inv_sqrt_d;
-          p.indices[base + j] = __float_as_int(sc);
-          m = fmaxf(m, sc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        __syncwarp();
-        int n = 0;
-        for (int jj = 0; jj <= jd; jj += 32) {
-          const int j = jj + lane;
-          const float sc = j <= jd ? __int_as_float(p.indices[base + j]) : -INFINITY;
-          __syncwarp();
-          const bool keep = j <= jd && (j == 0 || j == jd || sc - m >= p.log_tau);
-          const unsigned bal = __ballot_sync(0xffffffffu, keep);
-          if (keep) p.indices[base + n + __popc(bal & lt_mask)] = j;
-          n += __popc(bal);
-          __syncwarp();
-        }
-        if (lane == rr) p.counts[(long long)rh * NB + gb0 + ri] = n;
+        __syncthreads();
+        need_b = sm.need_b != 0;
       }
     }
-    if (fail && threadIdx.x == 0) dev_flag(p.dev_status, kDevTimeout);
+
+    if (is_row) {
+      if (!need_b) {
+        // every row keeps all of its causal blocks (or needs the exact pass): write 0..i
+        srch_write_all(rvalid && keep_all_row, rbase, rjd, p.indices, rcount);
+      } else if (rvalid && !exact_row) {
+        *rcount = sm.cnt[r];  // final after the last chunk's CTA barrier
+      }
+      if (sm.need_exact)
+        srch_exact_rows(rvalid && exact_row, rbase, rjd, p.q_pool + ((long long)(gb0 + ri) * p.hq + rh) * kHeadDim,
+                        p.k_pool, kb0, p.hkv, g, p.inv_sqrt_d, p.log_tau, p.indices, rcount);
+    }
     __syncthreads();  // the next tile reuses TMEM, the buffers and the flags
     if (__syncthreads_or(fail)) break;
   }
+  if (fail && threadIdx.x == 0) dev_flag(p.dev_status, kDevTimeout);
 
   if (is_mma) {
     // every issued MMA has completed before TMEM is released (own, generous limit: MMAs always finish)
