@@ -13,7 +13,8 @@ Entry points mirror the C ABI in include/fp.h:
     block_search_topp(...)  -> fp_block_search_topp (the cumulative top-p comparison selector)
     block_pool_search(...)  -> fp_block_pool_search (steps 1 + 2 fused)
     block_sparse_attn(...)  -> fp_block_sparse_attn
-    block_sparse_attn_fp8 / dense_attn_fp8 -> e4m3 Q / K attention (fp_*_fp8)
+    block_sparse_attn_fp8 / dense_attn_fp8 -> e4m3 Q / K attention, per-tensor scales (fp_*_fp8)
+    block_sparse_attn_fp8_blockscaled / dense_attn_fp8_blockscaled -> per-block power-of-two scales
     dense_attn(...)         -> fp_dense_attn
     sparse_prefill(...)     -> fp_sparse_prefill (all three steps, caller workspace)
     validate_lists(...)     -> fp_validate_lists
@@ -43,7 +44,8 @@ EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_poo
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version", "fp_paged_cache_init",
             "fp_paged_block_pool", "fp_paged_block_search", "fp_paged_block_sparse_attn", "fp_paged_dense_attn",
             "fp_paged_validate_lists", "fp_block_search_topp", "fp_block_sparse_attn_fp8", "fp_dense_attn_fp8",
-            "fp_index_buffer_elems", "fp_check_device_status")
+            "fp_index_buffer_elems", "fp_check_device_status", "fp_block_sparse_attn_fp8_blockscaled",
+            "fp_dense_attn_fp8_blockscaled")
 
 
 class FpError(RuntimeError):
@@ -77,6 +79,8 @@ def _load():
         "fp_block_search_topp": [P, vp, vp, f32, vp, vp, vp, vp, vp],
         "fp_block_sparse_attn_fp8": [P, vp, vp, vp, f32, f32, vp, vp, f32, vp, vp, vp, vp],
         "fp_dense_attn_fp8": [P, vp, vp, vp, f32, f32, f32, vp, vp, vp, vp],
+        "fp_block_sparse_attn_fp8_blockscaled": [P, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
+        "fp_dense_attn_fp8_blockscaled": [P, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
         "fp_paged_block_pool": [P, PC, vp, vp, vp, vp, vp],
         "fp_paged_block_search": [P, PC, vp, vp, f32, vp, vp, vp, vp],
         "fp_paged_block_sparse_attn": [P, PC, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp],
@@ -227,6 +231,22 @@ def dense_attn_fp8(p: Problem, q_e4m3, k_e4m3, v, q_scale: float, k_scale: float
                    dev_status=None, stream=None):
     _check(_lib.fp_dense_attn_fp8(p.ref, _ptr(q_e4m3), _ptr(k_e4m3), _ptr(v), float(q_scale), float(k_scale),
                                   float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
+def block_sparse_attn_fp8_blockscaled(p: Problem, q_e4m3, k_e4m3, v, q_exp, k_exp, counts, indices,
+                                      softmax_scale: float, out, lse=None, dev_status=None, stream=None):
+    """FP8 attention with per-block power-of-two scales: q_exp int8 [total_blocks, Hq], k_exp int8
+    [total_blocks, Hkv] (dequantised value = 2^exp * e4m3 code)."""
+    _check(_lib.fp_block_sparse_attn_fp8_blockscaled(p.ref, _ptr(q_e4m3), _ptr(k_e4m3), _ptr(v), _ptr(q_exp),
+                                                     _ptr(k_exp), _ptr(counts), _ptr(indices), float(softmax_scale),
+                                                     _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
+def dense_attn_fp8_blockscaled(p: Problem, q_e4m3, k_e4m3, v, q_exp, k_exp, softmax_scale: float, out, lse=None,
+                               dev_status=None, stream=None):
+    _check(_lib.fp_dense_attn_fp8_blockscaled(p.ref, _ptr(q_e4m3), _ptr(k_e4m3), _ptr(v), _ptr(q_exp), _ptr(k_exp),
+                                              float(softmax_scale), _ptr(out), _ptr(lse), _ptr(dev_status),
+                                              _stream(stream)))
 
 
 def dense_attn(p: Problem, q, k, v, softmax_scale: float, out, lse=None, dev_status=None, stream=None):

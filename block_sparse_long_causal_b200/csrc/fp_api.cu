@@ -133,7 +133,8 @@ uint64_t wait_limit_ns() {
 // softmax_scale * (qk_scale * q . k), qk_scale = q_scale * k_scale.
 fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* q, const void* k, const void* v,
                       const int32_t* counts, const int32_t* indices, int dense, float softmax_scale, void* out,
-                      float* lse, int32_t* dev_status, void* stream, bool fp8 = false, float qk_scale = 1.f) {
+                      float* lse, int32_t* dev_status, void* stream, bool fp8 = false, float qk_scale = 1.f,
+                      const int8_t* q_exp = nullptr, const int8_t* k_exp = nullptr) {
   fp_status st = check_problem(p);
   if (st != FP_OK) return st;
   if ((st = check_cache(p, c)) != FP_OK) return st;
@@ -167,6 +168,8 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   a.index_elems = index_elems(p, c);
   a.scale_log2 = scale * qk_scale * 1.4426950408889634f;
   a.fp8 = fp8 ? 1 : 0;
+  a.q_exp = q_exp;
+  a.k_exp = k_exp;
   a.sched = p->sched;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
@@ -437,6 +440,23 @@ fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q, const void* k, c
                      qk);
 }
 
+fp_status fp_block_sparse_attn_fp8_blockscaled(const fp_problem* p, const void* q, const void* k, const void* v,
+                                               const int8_t* q_exp, const int8_t* k_exp, const int32_t* counts,
+                                               const int32_t* indices, float softmax_scale, void* out, float* lse,
+                                               int32_t* dev_status, void* stream) {
+  if (!q_exp || !k_exp) return fail(FP_ERR_INVALID_ARG, "q_exp and k_exp must be non-NULL");
+  return attn_common(p, nullptr, q, k, v, counts, indices, 0, softmax_scale, out, lse, dev_status, stream, true, 1.f,
+                     q_exp, k_exp);
+}
+
+fp_status fp_dense_attn_fp8_blockscaled(const fp_problem* p, const void* q, const void* k, const void* v,
+                                        const int8_t* q_exp, const int8_t* k_exp, float softmax_scale, void* out,
+                                        float* lse, int32_t* dev_status, void* stream) {
+  if (!q_exp || !k_exp) return fail(FP_ERR_INVALID_ARG, "q_exp and k_exp must be non-NULL");
+  return attn_common(p, nullptr, q, k, v, nullptr, nullptr, 1, softmax_scale, out, lse, dev_status, stream, true, 1.f,
+                     q_exp, k_exp);
+}
+
 namespace {
 struct WorkspaceLayout {
   int64_t q_pool, k_pool, counts, indices, sched, total;  // byte offsets and total size
@@ -602,6 +622,6 @@ fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t
 
 const char* fp_last_error(void) { return g_err; }
 
-int32_t fp_version(void) { return 300; }
+int32_t fp_version(void) { return 400; }
 
 }  // extern "C"

@@ -46,7 +46,8 @@
 // TMA row comes from the block table and a query's causal limit is its key position (cached prefix
 // + local position); the plain prefill is compiled without it. kFp8 -- e4m3 Q and K: their tiles
 // are single 128-byte-row slabs loaded as uint8 boxes and Q K^T runs as kind::f8f6f4 (K = 32 per
-// MMA); V, P and O stay bf16 and the per-tensor scales are folded into the softmax scale.
+// MMA); V, P and O stay bf16. Per-tensor scales are folded into the softmax scale; per-block
+// power-of-two scales multiply it per row (query block) and per item (key block).
 #include "fp_internal.h"
 #include "fp_seq.cuh"
 
@@ -658,6 +659,13 @@ if (part == 3 && prev_part == 3) {
       // never take part in the warp's path votes, so a sequence's outputs do not depend on its
       // neighbours in the batch (or on what lies past the end of a cache page).
       const bool pad = qpos >= u.len;
+      // FP8 with per-block scales: this row's softmax scale times its query block's 2^q_exp; each item
+      // multiplies in its key block's 2^k_exp (plain prefill only: key block j is global block gb0 + j)
+      float row_sl2 = p.scale_log2;
+      if constexpr (kFp8) {
+        const int qblk = u.qt[slot] * (kTileM / BK) + half;
+        if (p.q_exp && active && qblk < u.nb) row_sl2 = ldexpf(p.scale_log2, (int)__ldg(p.q_exp + (long long)(u.gb0 + qblk) * p.hq + u.h[slot]));
+      }
       float m_run = -INFINITY, l_run = 0.f;
       int n = 0;
       while (true) {
@@ -667,13 +675,19 @@ if (part == 3 && prev_part == 3) {
         if (!active) continue;
         const int j = e >> 4, mask = e & 15;
         if (((mask >> (2 * slot)) & 3) == 0) continue;  // no list of this slot holds block j
+        int kexp = 0;
+        if constexpr (kFp8)
+          if (p.k_exp) kexp = __ldg(p.k_exp + (long long)(u.gb0 + j) * p.hkv + u.g);  // lands during the S wait
         // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
         if (__any_sync(kFull, !mbar_wait(b_s_full, cnt & 1, p.wait_limit_ns))) { fail = true; break; }
         tc_fence_after();
         // causal mask (diagonal tiles) and the list mask of this row's query block
         const int valid = ((mask >> mbit) & 1) ? (qpos - (j - (kCache ? u.pb : 0)) * BK) : -1;
         const bool masked = valid < BK - 1;
-        const uint64_t scale2 = f2_make(p.scale_log2, p.scale_log2);
+        float sl2 = row_sl2;  // this item's logits in log2 units per unit of S
+        if constexpr (kFp8)
+          if (p.k_exp) sl2 = ldexpf(row_sl2, kexp);
+        const uint64_t scale2 = f2_make(sl2, sl2);
         uint32_t pk[BK / 2];
         // Fast path, for unmasked items once the row has a reference max: no max pass. S streams
         // from TMEM in 32-column chunks (the next chunk loads while this one is exponentiated)
@@ -740,7 +754,7 @@ if (part == 3 && prev_part == 3) {
             }
             mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
           }
-          const float m_new = fmaxf(m_run, mx * p.scale_log2);
+          const float m_new = fmaxf(m_run, mx * sl2);
           // grow the reference max only when it rises by more than 2^8 (lazy rescale); the stale
           // max is exact because the numerator and the denominator share it
           const bool grow = m_new > m_run + 8.0f;

@@ -190,6 +190,26 @@ FP_API fp_status fp_dense_attn_fp8(const fp_problem* p, const void* q_e4m3, cons
                                    float q_scale, float k_scale, float softmax_scale, void* out, float* lse,
                                    int32_t* dev_status, void* stream);
 
+/* FP8 attention with per-block scales (FlashPrefill V2 abstract: FP8 inference): as
+ * fp_block_sparse_attn_fp8, but the dequantised value of q[t, h, :] is 2^q_exp[b, h] * code and of
+ * k[t, g, :] is 2^k_exp[b, g] * code, where b is the global block of token t (block_size tokens,
+ * restarting at every sequence, numbered as for the pooled tensors). q_exp: device int8
+ * [total_blocks, Hq]; k_exp: device int8 [total_blocks, Hkv]; exponents within [-64, 64]. Power-of-
+ * two scales, one per block and head (as in the microscaling formats), follow the range of each
+ * block's values while every dequantised value stays exact in bf16 and fp32. The logits are
+ * softmax_scale * 2^(q_exp + k_exp) * (q_code . k_code). NULL exponent arrays are invalid. */
+FP_API fp_status fp_block_sparse_attn_fp8_blockscaled(const fp_problem* p, const void* q_e4m3, const void* k_e4m3,
+                                                      const void* v, const int8_t* q_exp, const int8_t* k_exp,
+                                                      const int32_t* counts, const int32_t* indices,
+                                                      float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                                                      void* stream);
+
+/* Dense causal FP8 attention with per-block scales. */
+FP_API fp_status fp_dense_attn_fp8_blockscaled(const fp_problem* p, const void* q_e4m3, const void* k_e4m3,
+                                               const void* v, const int8_t* q_exp, const int8_t* k_exp,
+                                               float softmax_scale, void* out, float* lse, int32_t* dev_status,
+                                               void* stream);
+
 /* Bytes of workspace fp_sparse_prefill needs for this problem: the pooled Q and K, the counts, the
  * index lists and the attention's work counter (FP_SCHED_WORDS int32), each 256-byte aligned. */
 FP_API fp_status fp_sparse_prefill_workspace(const fp_problem* p, int64_t* bytes);

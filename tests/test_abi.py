@@ -197,6 +197,15 @@ def test_paged_calls_check_the_cache_and_arguments():
     assert fp._lib.fp_paged_block_pool(C.byref(p), C.byref(c), ok, ok, ok, ok, None) == fp.FP_ERR_INVALID_ARG
 
 
+def test_fp8_blockscaled_calls_reject_missing_exponents_before_launch():
+    st, p = _prob((0, 300), hq=4, hkv=2, B=128)
+    ok = C.c_void_p(4096)
+    assert fp._lib.fp_block_sparse_attn_fp8_blockscaled(C.byref(p), ok, ok, ok, None, ok, ok, ok, C.c_float(0.0), ok,
+                                                        None, None, None) == fp.FP_ERR_INVALID_ARG
+    assert fp._lib.fp_dense_attn_fp8_blockscaled(C.byref(p), ok, ok, ok, ok, None, C.c_float(0.0), ok, None, None,
+                                                 None) == fp.FP_ERR_INVALID_ARG
+
+
 def test_fp8_calls_reject_bad_scales_before_launch():
     st, p = _prob()
     ok = C.c_void_p(4096)
@@ -261,7 +270,7 @@ def test_check_device_status_maps_the_device_bits(bits, status, words):
 
 def test_struct_layouts_match_the_header(tmp_path):
     """ctypes mirrors of fp_problem and fp_paged_cache have the C sizes and offsets (the header
-    compiled by the host C compiler), and the ABI version is the one of this layout."""
+    compiled by the host C compiler), and the ABI version is at least the one of this layout."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
@@ -285,4 +294,4 @@ def test_struct_layouts_match_the_header(tmp_path):
         for f in fields[st]:
             assert int(got[f"{st} {f}"]) == getattr(cls, f).offset, (st, f)
     assert C.sizeof(fp.fp_problem) == 56 and C.sizeof(fp.fp_paged_cache) == 40
-    assert fp.version() == 300
+    assert fp.version() >= 300  # this layout of fp_problem (with sched) since 0.3.0
