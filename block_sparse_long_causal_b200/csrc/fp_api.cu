@@ -172,6 +172,7 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   a.k_exp = k_exp;
   a.sched = p->sched;
   a.out = static_cast<uint16_t*>(out);
+  a.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   a.lse = lse;
   a.dev_status = dev_status;
   a.wait_limit_ns = wait_limit_ns();

@@ -737,19 +737,18 @@ if (part == 3 && prev_part == 3) {
           float mx;
           {
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (masked) {
+            // keys past the row's causal limit (every key when its list lacks the block) become -inf
+            // here, and exact zeros below (MUFU ex2(-inf) = 0); one loop for masked and unmasked items
+            // keeps the kernel's code short (instruction-cache misses show in its stall profile)
 #pragma unroll
-              for (int c = 0; c < BK; ++c) {
-                const float v = (c <= valid) ? __uint_as_float(sr[c]) : -INFINITY;
-                sr[c] = __float_as_uint(v);
-                m4[c & 3] = fmaxf(m4[c & 3], v);
-              }
-            } else {
+            for (int c = 0; c < BK; c += 8) {
 #pragma unroll
-              for (int c = 0; c < BK; c += 8) {
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-                  m4[a] = fmax3(m4[a], __uint_as_float(sr[c + 2 * a]), __uint_as_float(sr[c + 2 * a + 1]));
+              for (int a = 0; a < 4; ++a) {
+                const float v0 = (c + 2 * a <= valid) ? __uint_as_float(sr[c + 2 * a]) : -INFINITY;
+                const float v1 = (c + 2 * a + 1 <= valid) ? __uint_as_float(sr[c + 2 * a + 1]) : -INFINITY;
+                sr[c + 2 * a] = __float_as_uint(v0);
+                sr[c + 2 * a + 1] = __float_as_uint(v1);
+                m4[a] = fmax3(m4[a], v0, v1);
               }
             }
             mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
@@ -786,28 +785,16 @@ if (part == 3 && prev_part == 3) {
           const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
           const uint64_t negm2 = f2_make(-m_use, -m_use);
           uint64_t sum2[2] = {0ull, 0ull};
-          if (masked) {
-            // exact zeros for masked keys: MUFU ex2(-inf) = 0
 #pragma unroll
-            for (int c = 0; c < BK; c += 2) {
-              float x0, x1;
-              f2_split(ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2), x0, x1);
-              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-              sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2_make(p0, p1));
-              pk[c / 2] = pack_bf16x2(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < BK; c += 2) {
-              const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
-              float x0, x1;
-              f2_split(x2, x0, x1);
-              const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
-              sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
-              float p0, p1;
-              f2_split(p2, p0, p1);
-              pk[c / 2] = pack_bf16x2(p0, p1);
-            }
+          for (int c = 0; c < BK; c += 2) {
+            const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
+            float p0, p1;
+            f2_split(p2, p0, p1);
+            pk[c / 2] = pack_bf16x2(p0, p1);
           }
           float a0, a1, b0, b1;
           f2_split(sum2[0], a0, a1);
@@ -851,11 +838,16 @@ if (part == 3 && prev_part == 3) {
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
         if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
-          dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+          if (p.out32) {  // 32-byte stores: a whole sector per thread and half the store instructions
+            st_global_v8(orow + c, w);
+            st_global_v8(orow + c + 16, w + 8);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
+            dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+          }
         }
       }
       if (row_ok && p.lse) {

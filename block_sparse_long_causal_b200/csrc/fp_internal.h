@@ -80,6 +80,7 @@ struct __align__(64) AttnParams {
   int64_t index_elems;
   float scale_log2;           // softmax_scale * log2(e)
   uint16_t* out;              // [T, Hq, d] bf16 bits
+  int32_t out32;              // out is 32-byte aligned: the epilogue stores 32 bytes per instruction
   float* lse;                 // [Hq, T] or null
   int32_t* dev_status;
   uint64_t wait_limit_ns;
