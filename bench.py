@@ -221,10 +221,11 @@ def supplementary(fp, p, sp, x, q, k, v, tau, stream, w, reps=3):
     out["fp8_attn_ms"] = round(ms8, 3)
     out["fp8_attn_tflops"] = round(eff1 / (ms8 * 1e-3) / 1e12, 2)
     out["fp8_note"] = "e4m3 Q K^T (kind::f8f6f4), bf16 P V; effective FLOPs of the kept blocks"
-    # the per-block power-of-two scale entry point on the same codes (all exponents 0: its work, one
-    # exponent load per query row and per item, does not depend on their values)
-    qe = torch.zeros((p.total_blocks, w.hq), dtype=torch.int8, device="cuda")
-    ke = torch.zeros((p.total_blocks, w.hkv), dtype=torch.int8, device="cuda")
+    # the per-block power-of-two scale entry point on the same codes, every block's exponent set to
+    # the power of two nearest the per-tensor scale (so the logits, and with them the softmax's path
+    # through the kernel, have the per-tensor run's magnitudes)
+    qe = torch.full((p.total_blocks, w.hq), int(round(math.log2(qs))), dtype=torch.int8, device="cuda")
+    ke = torch.full((p.total_blocks, w.hkv), int(round(math.log2(ks))), dtype=torch.int8, device="cuda")
     msb = timed(lambda: fp.block_sparse_attn_fp8_blockscaled(p, qc, kc, v, qe, ke, sp.counts, sp.indices, 0.0, o8,
                                                              None, sp.dev_status, stream))
     out["fp8_blockscaled_attn_ms"] = round(msb, 3)

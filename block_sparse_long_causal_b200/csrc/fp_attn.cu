@@ -74,6 +74,9 @@ constexpr int kUnitsEnd = -2;
 // Largest row sum of one item that the fast path (no max pass) accepts; see the softmax loop.
 constexpr float kFastSumLimit = 65536.f;
 
+// 2^e as a float for e in [-126, 127] (the per-block FP8 exponents lie in [-64, 64]): exact, so the
+// scaled logit equals ldexpf's
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 __device__ __forceinline__ uint32_t tmem_s(int k) { return 128u * k; }
 __device__ __forceinline__ uint32_t tmem_o(int k) { return 256u + 128u * k; }
 
@@ -664,7 +667,7 @@ if (part == 3 && prev_part == 3) {
       float row_sl2 = p.scale_log2;
       if constexpr (kFp8) {
         const int qblk = u.qt[slot] * (kTileM / BK) + half;
-        if (p.q_exp && active && qblk < u.nb) row_sl2 = ldexpf(p.scale_log2, (int)__ldg(p.q_exp + (long long)(u.gb0 + qblk) * p.hq + u.h[slot]));
+        if (p.q_exp && active && qblk < u.nb) row_sl2 = p.scale_log2 * pow2i(__ldg(p.q_exp + (long long)(u.gb0 + qblk) * p.hq + u.h[slot]));
       }
       float m_run = -INFINITY, l_run = 0.f;
       int n = 0;
@@ -686,7 +689,7 @@ if (part == 3 && prev_part == 3) {
         const bool masked = valid < BK - 1;
         float sl2 = row_sl2;  // this item's logits in log2 units per unit of S
         if constexpr (kFp8)
-          if (p.k_exp) sl2 = ldexpf(row_sl2, kexp);
+          if (p.k_exp) sl2 = row_sl2 * pow2i(kexp);
         const uint64_t scale2 = f2_make(sl2, sl2);
         uint32_t pk[BK / 2];
         // Fast path, for unmasked items once the row has a reference max: no max pass. S streams
