@@ -233,9 +233,6 @@ struct SrchSmem {                  // placed at a 1024-byte aligned address
   int need_b;                      // some row of the tile needs pass B
   int need_exact;                  // some row of the tile needs the exact pass
   int ok;
-  uint4 mask[kSrchRows];           // pass B: each row's keep masks of the current chunk (4 x 32 keys)
-  long long base[kSrchRows];       // each row's list start
-  int cnt[kSrchRows];              // each row's kept blocks so far
 };
 // Pooled-query staging at the start of a tile (in the key buffers, free then): 128 rows of 132 floats
 constexpr int kQStageStride = kHeadDim + 4;
@@ -387,23 +384,30 @@ __device__ __noinline__ float2 srch_pass_a(uint32_t scol, int j0, int jd, float 
 }
 
 // Rows, pass B: this row's keep mask of the chunk (acc >= thr, the sink, the diagonal, causal keys
-// only), then the warp writes its 32 rows' kept blocks, one row at a time, with coalesced stores.
-// masks / bases / cnts: the tile's per-row arrays in shared memory (shared addresses).
-__device__ __noinline__ void srch_pass_b(uint32_t scol, int j0, int jd, float thr, bool emit, uint32_t masks,
-                                         const long long* bases, int* cnts, int32_t* indices) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// only); then the warp writes the kept blocks of those of its 32 rows that have any in this chunk,
+// one row after another, with one coalesced store per 32 keys (the row's masks and list position
+// come from its lane by shuffles). rbase / row_n: this thread's row's list start and its blocks kept
+// so far; returns the new count.
+__device__ __noinline__ int srch_pass_b(uint32_t scol, int j0, int jd, float thr, bool emit, long long rbase,
+                                        int row_n, int32_t* indices) {
+  const int lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   uint32_t w[4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t a[32];
-    tmem_ld32(scol + 32 * q, a);  // warp-collective: every lane takes part
+  for (int h = 0; h < 2; ++h) {  // two 32-key loads in flight per wait
+    uint32_t a[2][32];
+    tmem_ld32(scol + 64 * h, a[0]);  // warp-collective: every lane takes part
+    tmem_ld32(scol + 64 * h + 32, a[1]);
     tmem_wait_ld();
-    reg_fence32(a);
-    uint32_t m = 0u;
+    reg_fence32(a[0]);
+    reg_fence32(a[1]);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) m |= (__uint_as_float(a[e]) >= thr ? 1u : 0u) << e;
-    w[q] = emit ? m : 0u;
+    for (int qq = 0; qq < 2; ++qq) {
+      uint32_t m = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) m |= (__uint_as_float(a[qq][e]) >= thr ? 1u : 0u) << e;
+      w[2 * h + qq] = emit ? m : 0u;
+    }
   }
   if (emit) {
     if (j0 == 0) w[0] |= 1u;                                                                // the sink
@@ -416,28 +420,22 @@ __device__ __noinline__ void srch_pass_b(uint32_t scol, int j0, int jd, float th
       else if (n < 32) w[q] &= (1u << n) - 1u;
     }
   }
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(masks + 16u * threadIdx.x), "r"(w[0]), "r"(w[1]),
-               "r"(w[2]), "r"(w[3])
-               : "memory");
-  __syncwarp();
-#pragma unroll 2
-  for (int rr = 0; rr < 32; ++rr) {
-    const int r2 = 32 * warp + rr;
-    uint4 m;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(m.x), "=r"(m.y), "=r"(m.z), "=r"(m.w) : "r"(masks + 16u * r2));
-    if ((m.x | m.y | m.z | m.w) == 0u) continue;
-    const long long base = bases[r2];
-    int n = cnts[r2];
-    const uint32_t words[4] = {m.x, m.y, m.z, m.w};
+  const long long mine = rbase + row_n;
+  unsigned todo = __ballot_sync(0xffffffffu, (w[0] | w[1] | w[2] | w[3]) != 0u);
+  while (todo) {
+    const int rr = __ffs(todo) - 1;
+    todo &= todo - 1;
+    const long long b = (long long)(((unsigned long long)__shfl_sync(0xffffffffu, (unsigned)(mine >> 32), rr) << 32) |
+                                    (unsigned)__shfl_sync(0xffffffffu, (unsigned)mine, rr));
+    int n = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      if ((words[q] >> lane) & 1u) indices[base + n + __popc(words[q] & lt_mask)] = j0 + 32 * q + lane;
-      n += __popc(words[q]);
+      const uint32_t m = __shfl_sync(0xffffffffu, w[q], rr);
+      if ((m >> lane) & 1u) indices[b + n + __popc(m & lt_mask)] = j0 + 32 * q + lane;
+      n += __popc(m);
     }
-    __syncwarp();
-    if (lane == 0) cnts[r2] = n;
   }
-  __syncwarp();
+  return row_n + __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]);
 }
 
 // Rows of a tile that keeps every causal block: the warp writes 0..jd of each such row of its 32.
@@ -533,7 +531,6 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
   const uint32_t kstage = smem_u32(&sm.kstage[0][0]);
   const uint32_t kbuf0 = smem_u32(sm.k[0]), kbuf1 = smem_u32(sm.k[1]);
   const uint32_t bar0 = smem_u32(&sm.bar_s[0]), bar1 = smem_u32(&sm.bar_s[1]);
-  const uint32_t masks = smem_u32(&sm.mask[0]);
   uint32_t uses0 = 0u, uses1 = 0u;                   // completions of bar_s[0] / bar_s[1] waited on so far
   bool fail = false;
 
@@ -566,10 +563,7 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
       sm.need_b = 0;
       sm.need_exact = 0;
     }
-    if (is_row) {
-      sm.base[r] = rbase;
-      sm.cnt[r] = 0;
-    }
+    int row_n = 0;  // pass B: this row's kept blocks so far
     if (is_row && !p.keep_all) {
       // the pooled queries of this warp's 32 rows: coalesced row copies into the staging area, then
       // each thread splits its own row into bf16 hi + lo and stores both into TMEM (the A operand of
@@ -649,7 +643,7 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
             mx = v.x;
             mn = v.y;
           } else {
-            srch_pass_b(scol, c * kSrchKeys, rjd, thr, rvalid && !exact_row, masks, sm.base, sm.cnt, p.indices);
+            row_n = srch_pass_b(scol, c * kSrchKeys, rjd, thr, rvalid && !exact_row, rbase, row_n, p.indices);
           }
           tc_fence_before();
         }
@@ -682,7 +676,7 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
         // every row keeps all of its causal blocks (or needs the exact pass): write 0..i
         srch_write_all(rvalid && keep_all_row, rbase, rjd, p.indices, rcount);
       } else if (rvalid && !exact_row) {
-        *rcount = sm.cnt[r];  // final after the last chunk's CTA barrier
+        *rcount = row_n;
       }
       if (sm.need_exact)
         srch_exact_rows(rvalid && exact_row, rbase, rjd, p.q_pool + ((long long)(gb0 + ri) * p.hq + rh) * kHeadDim,
