@@ -44,7 +44,7 @@ EXPORTED = ("fp_problem_init", "fp_block_pool", "fp_block_search", "fp_block_poo
             "fp_validate_lists", "fp_selftest_exp2", "fp_last_error", "fp_version", "fp_paged_cache_init",
             "fp_paged_block_pool", "fp_paged_block_search", "fp_paged_block_sparse_attn", "fp_paged_dense_attn",
             "fp_paged_validate_lists", "fp_block_search_topp", "fp_block_sparse_attn_fp8", "fp_dense_attn_fp8",
-            "fp_index_buffer_elems", "fp_check_device_status", "fp_block_sparse_attn_fp8_blockscaled",
+            "fp_index_buffer_elems", "fp_check_device_status", "fp_key_split_bytes", "fp_block_sparse_attn_fp8_blockscaled",
             "fp_dense_attn_fp8_blockscaled")
 
 
@@ -58,7 +58,8 @@ class fp_problem(C.Structure):
     _fields_ = [("cu_seqlens", C.c_void_p), ("num_seqs", C.c_int32), ("total_tokens", C.c_int32),
                 ("total_blocks", C.c_int32), ("max_seq_blocks", C.c_int32), ("index_elems", C.c_int64),
                 ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
-                ("block_size", C.c_int32), ("sched", C.c_void_p)]
+                ("block_size", C.c_int32), ("sched", C.c_void_p), ("key_split", C.c_void_p),
+                ("key_split_bytes", C.c_int64)]
 
 
 class fp_paged_cache(C.Structure):
@@ -99,6 +100,7 @@ def _load():
         "fp_sparse_prefill_noalloc": [P, vp, vp, vp, f32, f32, vp, vp, vp, vp],
         "fp_index_buffer_elems": [vp, i32, i32, i32, C.POINTER(C.c_int64)],
         "fp_check_device_status": [i32],
+        "fp_key_split_bytes": [P, vp, C.POINTER(C.c_int64)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -145,10 +147,12 @@ class Problem:
     """fp_problem plus the device tensors it points to (kept alive here): cu_seqlens and, with
     work_counter (the default on a CUDA device), the attention calls' work counter -- zeroed once,
     left at zero by every launch, so launches of this problem must be ordered (one stream, or
-    events); give concurrent streams one Problem each."""
+    events); give concurrent streams one Problem each. With key_split (the default on a CUDA device)
+    the searches of the plain problem split the pooled keys once per call into a scratch buffer held
+    here (fp_problem.key_split)."""
 
     def __init__(self, cu_seqlens_host, cu_seqlens_dev: torch.Tensor, num_q_heads: int, num_kv_heads: int,
-                 head_dim: int, block_size: int, work_counter: bool = True):
+                 head_dim: int, block_size: int, work_counter: bool = True, key_split: bool = True):
         host = np.ascontiguousarray(cu_seqlens_host, np.int32)
         if cu_seqlens_dev.dtype != torch.int32:
             raise ValueError("cu_seqlens must be int32")
@@ -161,6 +165,12 @@ class Problem:
         if work_counter and cu_seqlens_dev.is_cuda:
             self.sched = torch.zeros(FP_SCHED_WORDS, dtype=torch.int32, device=cu_seqlens_dev.device)
             self.c.sched = self.sched.data_ptr()
+        self.key_split = None
+        if key_split and cu_seqlens_dev.is_cuda:
+            nbytes = key_split_bytes(self)
+            self.key_split = torch.empty(nbytes, dtype=torch.uint8, device=cu_seqlens_dev.device)
+            self.c.key_split = self.key_split.data_ptr()
+            self.c.key_split_bytes = nbytes
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)
@@ -171,10 +181,22 @@ class Problem:
 
 
 def problem(cu_seqlens_host, num_q_heads: int, num_kv_heads: int, head_dim: int = 128, block_size: int = 128,
-            device="cuda", work_counter: bool = True) -> Problem:
+            device="cuda", work_counter: bool = True, key_split: bool = True) -> Problem:
     host = np.ascontiguousarray(cu_seqlens_host, np.int32)
     dev = torch.from_numpy(host.copy()).to(device)
-    return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size, work_counter)
+    return Problem(host, dev, num_q_heads, num_kv_heads, head_dim, block_size, work_counter, key_split)
+
+
+def _cache_ref(cache):
+    return cache.ref if isinstance(cache, PagedCache) else C.byref(cache)
+
+
+def key_split_bytes(p, cache=None) -> int:
+    """fp_key_split_bytes: bytes of the search's key split scratch for this problem (and paged cache)."""
+    n = C.c_int64(0)
+    ref = p.ref if isinstance(p, Problem) else C.byref(p)
+    _check(_lib.fp_key_split_bytes(ref, None if cache is None else _cache_ref(cache), C.byref(n)))
+    return int(n.value)
 
 
 def index_buffer_elems(seqlens, block_size: int, num_q_heads: int) -> int:
@@ -300,6 +322,14 @@ class PagedCache:
         _check(_lib.fp_paged_cache_init(C.byref(self.c), p.ref, p.cu_host.ctypes.data_as(C.c_void_p),
                                         pre.ctypes.data_as(C.c_void_p), _ptr(prefix_lens_dev), _ptr(self.table_dev),
                                         int(self.table_dev.shape[1]), int(page_size), int(num_pages)))
+        # the paged search's key split covers the cached prefixes' key blocks too
+        self.key_split = None
+        if p.key_split is not None:
+            nbytes = key_split_bytes(p, self)
+            self.key_split = torch.empty(nbytes, dtype=torch.uint8, device=prefix_lens_dev.device)
+            self.search_problem = fp_problem.from_buffer_copy(p.c)
+            self.search_problem.key_split = self.key_split.data_ptr()
+            self.search_problem.key_split_bytes = nbytes
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)
@@ -323,7 +353,8 @@ def paged_block_pool(p: Problem, c: PagedCache, q, k_cache, q_pool, k_pool, stre
 
 def paged_block_search(p: Problem, c: PagedCache, q_pool, k_pool, tau: float, counts, indices, dev_status=None,
                        stream=None):
-    _check(_lib.fp_paged_block_search(p.ref, c.ref, _ptr(q_pool), _ptr(k_pool), float(tau), _ptr(counts),
+    ref = C.byref(c.search_problem) if c.key_split is not None and p is c.p else p.ref
+    _check(_lib.fp_paged_block_search(ref, c.ref, _ptr(q_pool), _ptr(k_pool), float(tau), _ptr(counts),
                                       _ptr(indices), _ptr(dev_status), _stream(stream)))
 
 

@@ -366,12 +366,33 @@ fp_status search_impl(const fp_problem* p, const fp_paged_cache* c, const float*
     return fail(FP_ERR_INVALID_ARG, "q_pool, k_pool, counts and indices must be non-NULL");
   if (!aligned16(q_pool) || !aligned16(k_pool)) return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
   if (!std::isfinite(tau)) return fail(FP_ERR_INVALID_ARG, "tau must be finite");
+  const fp::KeySplitLayout kl = fp::key_split_layout(seq_info(p, c).total_kv_blocks, p->num_kv_heads);
+  if (p->key_split) {
+    if ((reinterpret_cast<uintptr_t>(p->key_split) & 255u) != 0)
+      return fail(FP_ERR_INVALID_ARG, "problem.key_split must be 256-byte aligned");
+    if (p->key_split_bytes < kl.total)
+      return fail(FP_ERR_INVALID_ARG, "problem.key_split holds %lld bytes, this search needs %lld",
+                  (long long)p->key_split_bytes, (long long)kl.total);
+  }
   if (p->total_blocks == 0) return FP_OK;
   fp::SearchParams a = search_params(p, c, tau, k_pool, counts, indices, dev_status);
   a.q_pool = q_pool;
+  if (p->key_split) {
+    a.ksplit = static_cast<unsigned char*>(p->key_split);
+    a.knorm2 = reinterpret_cast<float*>(static_cast<unsigned char*>(p->key_split) + kl.norms);
+  }
   return cuda_status(fp::launch_search(a, static_cast<cudaStream_t>(stream)), "search launch");
 }
 }  // namespace
+
+fp_status fp_key_split_bytes(const fp_problem* p, const fp_paged_cache* cache, int64_t* bytes) {
+  fp_status st = check_problem(p);
+  if (st != FP_OK) return st;
+  if ((st = check_cache(p, cache)) != FP_OK) return st;
+  if (!bytes) return fail(FP_ERR_INVALID_ARG, "bytes must be non-NULL");
+  *bytes = fp::key_split_layout(seq_info(p, cache).total_kv_blocks, p->num_kv_heads).total;
+  return FP_OK;
+}
 
 fp_status fp_block_search(const fp_problem* p, const float* q_pool, const float* k_pool, float tau,
                           int32_t* counts, int32_t* indices, int32_t* dev_status, void* stream) {
@@ -460,7 +481,7 @@ fp_status fp_dense_attn_fp8_blockscaled(const fp_problem* p, const void* q, cons
 
 namespace {
 struct WorkspaceLayout {
-  int64_t q_pool, k_pool, counts, indices, sched, total;  // byte offsets and total size
+  int64_t q_pool, k_pool, counts, indices, sched, ksplit, total;  // byte offsets and total size
 };
 int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
 WorkspaceLayout workspace_layout(const fp_problem* p) {
@@ -471,7 +492,8 @@ WorkspaceLayout workspace_layout(const fp_problem* p) {
   w.counts = align256(w.k_pool + nb * p->num_kv_heads * d * 4);
   w.indices = align256(w.counts + (int64_t)p->num_q_heads * nb * 4);
   w.sched = align256(w.indices + p->index_elems * 4);
-  w.total = align256(w.sched + FP_SCHED_WORDS * 4);
+  w.ksplit = align256(w.sched + FP_SCHED_WORDS * 4);
+  w.total = w.ksplit + fp::key_split_layout(nb, p->num_kv_heads).total;
   return w;
 }
 }  // namespace
@@ -503,11 +525,13 @@ fp_status fp_sparse_prefill(const fp_problem* p, const void* q, const void* k, c
   // the work counter lives in the workspace (scratch between calls): zeroed here, in stream order
   fp_problem pw = *p;
   pw.sched = reinterpret_cast<int32_t*>(base + w.sched);
+  pw.key_split = base + w.ksplit;
+  pw.key_split_bytes = w.total - w.ksplit;
   if ((st = cuda_status(cudaMemsetAsync(pw.sched, 0, FP_SCHED_WORDS * sizeof(int32_t),
                                         static_cast<cudaStream_t>(stream)), "work counter reset")) != FP_OK)
     return st;
   if ((st = fp_block_pool(p, q, k, q_pool, k_pool, stream)) != FP_OK) return st;
-  if ((st = fp_block_search(p, q_pool, k_pool, tau, counts, indices, dev_status, stream)) != FP_OK) return st;
+  if ((st = fp_block_search(&pw, q_pool, k_pool, tau, counts, indices, dev_status, stream)) != FP_OK) return st;
   return fp_block_sparse_attn(&pw, q, k, v, counts, indices, softmax_scale, out, lse, dev_status, stream);
 }
 
@@ -623,6 +647,6 @@ fp_status fp_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t
 
 const char* fp_last_error(void) { return g_err; }
 
-int32_t fp_version(void) { return 400; }
+int32_t fp_version(void) { return 500; }
 
 }  // extern "C"

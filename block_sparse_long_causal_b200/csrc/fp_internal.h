@@ -56,7 +56,24 @@ struct SearchParams {
   int64_t index_elems;
   int32_t* dev_status;
   uint64_t wait_limit_ns;     // limit of every bounded wait of the search kernel
+  // optional key split (null: each tile splits the keys it reads): row (key block kb, kv-head g) at
+  // ksplit + (kb * hkv + g) * kKeySplitRow holds bf16 hi of the 128 dims, then bf16 lo; knorm2 the
+  // row's |kbar|^2; both written by the split kernel at the start of the search launch
+  unsigned char* ksplit;
+  float* knorm2;
 };
+
+constexpr int64_t kKeySplitRow = 512;  // bytes per (key block, kv-head): 128 bf16 hi + 128 bf16 lo
+// Layout of the key split buffer for nbk key blocks: split rows, then (256-byte aligned) the norms.
+struct KeySplitLayout {
+  int64_t norms, total;
+};
+inline KeySplitLayout key_split_layout(int64_t nbk, int64_t hkv) {
+  KeySplitLayout l;
+  l.norms = (nbk * hkv * kKeySplitRow + 255) & ~(int64_t)255;
+  l.total = (l.norms + nbk * hkv * 4 + 255) & ~(int64_t)255;
+  return l;
+}
 
 struct ValidateParams {
   SeqInfo seq;

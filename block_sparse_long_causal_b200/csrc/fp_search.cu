@@ -279,6 +279,52 @@ __device__ __forceinline__ void cp_async16_s(uint32_t dst, const void* src, bool
 // The role code of the search kernel, one copy each (not inlined): the kernel's 9 warps run three
 // different instruction streams, and a small hot footprint keeps them in the instruction cache.
 
+// Key split (optional scratch, one launch before the search kernel): every pooled key row (key block
+// kb, kv-head g) once, as bf16 hi + lo of its 128 dims (the same split the converters make) and its
+// |kbar|^2; one warp per row, lane l holding dims 4l .. 4l + 3.
+__global__ void __launch_bounds__(256) ksplit_kernel(const float* __restrict__ k_pool, int64_t rows,
+                                                     unsigned char* __restrict__ ksplit, float* __restrict__ knorm2) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += nwarps) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(k_pool + row * kHeadDim) + lane);
+    const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+    const uint32_t l01 = pack_bf16x2(v.x - __uint_as_float(h01 << 16), v.y - __uint_as_float(h01 & 0xffff0000u));
+    const uint32_t l23 = pack_bf16x2(v.z - __uint_as_float(h23 << 16), v.w - __uint_as_float(h23 & 0xffff0000u));
+    unsigned char* dst = ksplit + row * kKeySplitRow + 8 * lane;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(dst + 256) = make_uint2(l01, l23);
+    // |kbar|^2 in the converters' order: per lane fma chain, then the lane sums of 4-lane groups, then
+    // the 8 group sums as a butterfly (the same value on every lane)
+    float n2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+    if (lane == 0) knorm2[row] = n2;
+  }
+}
+
+// Converters, with a key split: copy the split rows of chunk cc straight into the swizzled key tiles at
+// kbuf (lane l < 16: 16 bytes of hi, dims 8l .. 8l + 7; lane l >= 16: the same of lo), zeros past the
+// tile's last causal key. Returns the largest |kbar|^2 of the chunk's valid keys this lane read.
+__device__ __noinline__ float srch_copy_split(uint32_t kbuf, const unsigned char* ksplit, const float* knorm2, int hkv,
+                                              int g, int kb0, int jmax, int cc) {
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 4;
+  const uint32_t piece = lane & 15;
+  const uint32_t dst0 = kbuf + ((lane >> 4) ? kKTile : 0u) + (piece >> 3) * kKSlab;
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) {
+    const int jr = cw + 4 * i;
+    const int j = cc * kSrchKeys + jr;
+    const bool valid = j <= jmax;
+    const long long row = (long long)(kb0 + (valid ? j : 0)) * hkv + g;
+    cp_async16_s(dst0 + jr * 128 + (((piece & 7) ^ (uint32_t)(jr & 7)) << 4), ksplit + row * kKeySplitRow + 16 * lane,
+                 valid);
+  }
+  cp_async_commit();
+  const int j = cc * kSrchKeys + cw + 4 * lane;  // lane l reads the norm of key row cw + 4 l
+  return j <= jmax ? __ldg(knorm2 + (long long)(kb0 + j) * hkv + g) : 0.f;
+}
+
 // Converters: copy this thread's share of the fp32 pooled keys of chunk cc into the staging area:
 // converter warp cw takes keys cw, cw + 4, ..., lane l the 16 bytes at dims 4l..4l+3 of each
 // (coalesced). A thread later converts exactly the bytes it copied.
@@ -609,13 +655,19 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
     for (int pass = p.keep_all ? 2 : 0; pass < 2; ++pass) {
       if (pass == 1 && !need_b) break;
       if (is_conv) {
-        srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 0);
-        kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf0));
-        if (nch > 1) {
-          srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 1);
-          kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf1));
+        if (p.ksplit) {  // split keys: chunks 0 and 1 copied straight into the two key buffers
+          kmax2 = fmaxf(kmax2, srch_copy_split(kbuf0, p.ksplit, p.knorm2, p.hkv, g, kb0, jmax, 0));
+          if (nch > 1) kmax2 = fmaxf(kmax2, srch_copy_split(kbuf1, p.ksplit, p.knorm2, p.hkv, g, kb0, jmax, 1));
+          cp_async_wait_all();
+        } else {
+          srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 0);
+          kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf0));
+          if (nch > 1) {
+            srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 1);
+            kmax2 = fmaxf(kmax2, srch_convert(kstage, kbuf1));
+          }
+          if (nch > 2) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 2);  // lands while the first chunks are scored
         }
-        if (nch > 2) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, 2);  // lands while the first chunks are scored
         fence_proxy_async_smem();
       }
       __syncthreads();
@@ -648,8 +700,13 @@ __global__ void __launch_bounds__(kSrchThreads, 1) search_kernel(const SearchPar
           tc_fence_before();
         }
         if (is_conv && c + 2 < nch) {
-          kmax2 = fmaxf(kmax2, srch_convert(kstage, b ? kbuf1 : kbuf0));  // chunk c + 2, staged during chunk c + 1
-          if (c + 3 < nch) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, c + 3);
+          if (p.ksplit) {  // chunk c + 2 into the buffer that chunk c's MMAs have released
+            kmax2 = fmaxf(kmax2, srch_copy_split(b ? kbuf1 : kbuf0, p.ksplit, p.knorm2, p.hkv, g, kb0, jmax, c + 2));
+            cp_async_wait_all();
+          } else {
+            kmax2 = fmaxf(kmax2, srch_convert(kstage, b ? kbuf1 : kbuf0));  // chunk c + 2, staged during chunk c + 1
+            if (c + 3 < nch) srch_stage(kstage, p.k_pool, p.hkv, g, kb0, jmax, c + 3);
+          }
           fence_proxy_async_smem();
         }
         __syncthreads();
@@ -713,6 +770,12 @@ cudaError_t launch_search(const SearchParams& sp, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(tiles < sms ? tiles : sms);
   if (grid <= 0) return cudaSuccess;
+  if (p.ksplit) {  // every pooled key split once, before the tiles read them
+    const int64_t rows = (int64_t)p.seq.total_kv_blocks * p.hkv;
+    const int64_t blocks = (rows + 7) / 8;
+    ksplit_kernel<<<(int)(blocks < 8 * sms ? blocks : 8 * sms), 256, 0, st>>>(p.k_pool, rows, p.ksplit, p.knorm2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   search_kernel<<<grid, kSrchThreads, srch_smem_bytes(p.seq.num_seqs), st>>>(p);
   return cudaGetLastError();
 }

@@ -84,6 +84,9 @@ typedef struct fp_problem {
   int32_t head_dim;          /* d; 128 is supported */
   int32_t block_size;        /* B; 64 or 128 */
   int32_t* sched;            /* optional work counter of the attention calls, see below; NULL after init */
+  void* key_split;           /* optional search scratch (the pooled keys split for the tensor cores), see
+                                below; NULL after init */
+  int64_t key_split_bytes;   /* its size in bytes */
 } fp_problem;
 
 /* Work counter. fp_problem_init leaves sched NULL: an attention launch then gives each CTA a fixed
@@ -95,6 +98,19 @@ typedef struct fp_problem {
  * streams, no ordering between them) must not share them. The results are identical either way.
  * fp_sparse_prefill(_noalloc) use words inside their workspace and ignore sched. */
 #define FP_SCHED_WORDS 2
+
+/* Key split. The block search scores pooled keys on the tensor cores as bf16 hi + lo halves (step 2
+ * below). fp_problem_init leaves key_split NULL: each search tile then splits the pooled keys it reads
+ * itself (every tile of a kv-head splits the same keys again). A caller may point key_split at
+ * key_split_bytes >= fp_key_split_bytes(p, cache) bytes of device memory (256-byte aligned, contents
+ * scratch): fp_block_search (and the fused and paged searches) then split every pooled key once per
+ * call, into that buffer, before the search kernel reads them. The lists are the same either way
+ * (the split and the error bound of each key are). Calls that may run at the same time must not share
+ * the buffer. cache: NULL for the plain problem, or the paged-cache description the search will use
+ * (whose pooled keys include the cached prefixes). fp_sparse_prefill(_noalloc) keep theirs in the
+ * workspace. Host-only. */
+struct fp_paged_cache;
+FP_API fp_status fp_key_split_bytes(const fp_problem* p, const struct fp_paged_cache* cache, int64_t* bytes);
 
 /* Length, in int32 entries, of the index buffer of a problem: sum_s Hq * nb_s (nb_s + 1) / 2 with
  * nb_s = ceil(L_s / block_size) (the triangular layout above: query block i of a sequence keeps at

@@ -125,7 +125,8 @@ def test_sparse_prefill_workspace_and_argument_checks():
     assert fp._lib.fp_sparse_prefill_workspace(C.byref(p), C.byref(n)) == fp.FP_OK
     nb = 3 + 1 + 4
     need = 0
-    for nbytes in (nb * 4 * 128 * 4, nb * 2 * 128 * 4, 4 * nb * 4, p.index_elems * 4, fp.FP_SCHED_WORDS * 4):
+    for nbytes in (nb * 4 * 128 * 4, nb * 2 * 128 * 4, 4 * nb * 4, p.index_elems * 4, fp.FP_SCHED_WORDS * 4,
+                   nb * 2 * 512, nb * 2 * 4):  # ..., the work counter, the key split rows and their norms
         need += (nbytes + 255) // 256 * 256
     assert n.value == need
     ok, null = C.c_void_p(4096), None
@@ -293,5 +294,31 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert int(got[f"{st} size"]) == C.sizeof(cls)
         for f in fields[st]:
             assert int(got[f"{st} {f}"]) == getattr(cls, f).offset, (st, f)
-    assert C.sizeof(fp.fp_problem) == 56 and C.sizeof(fp.fp_paged_cache) == 40
-    assert fp.version() >= 300  # this layout of fp_problem (with sched) since 0.3.0
+    assert C.sizeof(fp.fp_problem) == 72 and C.sizeof(fp.fp_paged_cache) == 40
+    assert fp.version() >= 500  # this layout of fp_problem (with sched, key_split) since 0.5.0
+
+
+def test_key_split_sizes_and_checks():
+    """fp_key_split_bytes: 512 bytes (bf16 hi + lo of 128 dims) and one float per (key block, kv-head),
+    each part 256-byte aligned; the paged size counts the cached prefixes' key blocks. A search whose
+    key_split is misaligned or too small is refused on the host, before any launch."""
+    st, p = _prob((0, 300, 301, 700), hq=4, hkv=2, B=128)
+    assert st == fp.FP_OK
+    n = C.c_int64(0)
+    assert fp._lib.fp_key_split_bytes(C.byref(p), None, C.byref(n)) == fp.FP_OK
+    nb = 3 + 1 + 4
+    rup = lambda x: (x + 255) // 256 * 256
+    assert n.value == rup(nb * 2 * 512) + rup(nb * 2 * 4)
+    assert fp._lib.fp_key_split_bytes(C.byref(p), None, None) == fp.FP_ERR_INVALID_ARG
+    st, pp, c = _paged(cu=(0, 300, 500), prefixes=(256, 0))
+    assert st == fp.FP_OK
+    assert fp._lib.fp_key_split_bytes(C.byref(pp), C.byref(c), C.byref(n)) == fp.FP_OK
+    nbk = (256 + 300 + 127) // 128 + (200 + 127) // 128
+    assert n.value == rup(nbk * 2 * 512) + rup(nbk * 2 * 4)
+    ok = C.c_void_p(4096)
+    need = rup(nb * 2 * 512) + rup(nb * 2 * 4)
+    search = lambda: fp._lib.fp_block_search(C.byref(p), ok, ok, C.c_float(0.5), ok, ok, None, None)
+    p.key_split, p.key_split_bytes = 4096 + 16, need
+    assert search() == fp.FP_ERR_INVALID_ARG and "key_split" in _err()
+    p.key_split, p.key_split_bytes = 4096, need - 1
+    assert search() == fp.FP_ERR_INVALID_ARG and "key_split" in _err()

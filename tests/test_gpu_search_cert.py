@@ -17,7 +17,7 @@ import pytest
 
 import oracle
 import synth
-from helpers import compare_lists, to_dev
+from helpers import compare_lists, keep_mask, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +72,8 @@ def _tau_near_many_blocks(qb, kb, cu, B, hq):
     ("exact rows", 10.0, 3.0, 0.0015),
 ])
 @pytest.mark.parametrize("B", [64, 128])
-def test_lists_exact_just_outside_the_tie_band(name, q_norm, c_norm, e_sigma, B):
+@pytest.mark.parametrize("key_split", [True, False], ids=["key_split", "tile_split"])
+def test_lists_exact_just_outside_the_tie_band(name, q_norm, c_norm, e_sigma, B, key_split):
     import torch
     import block_sparse_long_causal_b200 as fp
     nb, hq, hkv = 200, 4, 2
@@ -82,10 +83,39 @@ def test_lists_exact_just_outside_the_tie_band(name, q_norm, c_norm, e_sigma, B)
     tau, near = _tau_near_many_blocks(qb, kb, cu, B, hq)
     assert near >= 200, near  # the case has teeth: many blocks sit just outside the band
     oc, oi, band = oracle.search(qb, kb, cu, B, tau)
-    p = fp.problem(cu, hq, hkv, 128, B)
+    p = fp.problem(cu, hq, hkv, 128, B, key_split=key_split)
+    assert (p.key_split is not None) == key_split
     sp = fp.SparsePrefill(p)
     sp.search(to_dev(x["q"]), to_dev(x["k"]), tau)
     torch.cuda.synchronize()
     assert int(sp.dev_status.item()) == 0
     np.testing.assert_allclose(sp.k_pool[:nb].cpu().numpy(), kb, rtol=0, atol=1e-6)
     compare_lists(sp.counts.cpu().numpy(), sp.indices[: p.index_elems].cpu().numpy(), oc, oi, band, cu, B, hq)
+
+
+@pytest.mark.parametrize("lens,hq,hkv,B,tau", [
+    ((1000,), 4, 2, 128, 0.9),
+    ((257, 1, 130, 640), 8, 2, 128, 0.7),
+    ((700, 129), 4, 2, 64, 0.5),
+    ((900, 385), 6, 2, 128, 0.6),      # G = 3
+    ((2000,), 16, 2, 64, 0.95),        # G = 8
+    ((3000,), 2, 2, 128, 0.05),        # every row certified all-kept
+])
+def test_key_split_and_tile_split_give_the_same_lists(lens, hq, hkv, B, tau):
+    """The searches that split the pooled keys once per call (fp_problem.key_split) and per tile give
+    the same lists bit for bit: same split, same error bound per key, same decisions."""
+    import torch
+    import block_sparse_long_causal_b200 as fp
+    x = synth.random_inputs(lens, hq, hkv, 128, seed=sum(lens) + hq, scale=1.0)
+    cu = x["cu_seqlens"]
+    out = []
+    for ks in (True, False):
+        p = fp.problem(cu, hq, hkv, 128, B, key_split=ks)
+        sp = fp.SparsePrefill(p)
+        sp.search(to_dev(x["q"]), to_dev(x["k"]), tau)
+        torch.cuda.synchronize()
+        assert int(sp.dev_status.item()) == 0
+        out.append((sp.counts.cpu().numpy().copy(), sp.indices[: p.index_elems].cpu().numpy().copy()))
+    np.testing.assert_array_equal(out[0][0], out[1][0])
+    # the lists (entries past a row's count are scratch of the exact pass, compared through the masks)
+    np.testing.assert_array_equal(keep_mask(out[0][0], out[0][1], cu, B, hq), keep_mask(out[1][0], out[1][1], cu, B, hq))
