@@ -482,7 +482,8 @@ def run_ours(args):
                      "traffic": measured_traffic(f"attn_kernel<{w.block}>", w.name)},
         "search_roofline": None,
         "sparse_settings": sparse_settings,
-        "gpu_launches": 3 * args.steps,
+        # per step: pool_kernel, (ksplit_kernel with the problem's key split,) search_kernel, attn_kernel
+        "gpu_launches": (4 if p.key_split is not None else 3) * args.steps,
         "supplementary": supp,
         "dev_status": status,
         "clocks": clk,
