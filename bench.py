@@ -483,7 +483,8 @@ def run_ours(args):
         "search_roofline": None,
         "sparse_settings": sparse_settings,
         # per step: pool_kernel, (ksplit_kernel with the problem's key split,) search_kernel, attn_kernel
-        "gpu_launches": (4 if p.key_split is not None else 3) * args.steps,
+        # and, for B = 128, attn_rows_kernel (one of the two attention kernels returns at once)
+        "gpu_launches": (3 + (p.key_split is not None) + (w.block == 128)) * args.steps,
         "supplementary": supp,
         "dev_status": status,
         "clocks": clk,

@@ -40,6 +40,10 @@
 // (fp_problem.sched) each CTA takes the next untaken unit of that order when its producer is free,
 // which keeps the grid balanced for lists of any lengths (a load model of the 128K workload puts
 // the busiest SM of a fixed share 4-15% above the mean, more the sparser the lists).
+// A second schedule, for sparse lists (plain bf16 prefill, B = 128; see "row schedule" below), runs
+// one query tile per unit with both softmax warpgroups on the same tile, each on half of every
+// item's keys, and alternates two S buffers between items; the kernel picks it when fewer than 40% of
+// the causal blocks are kept.
 // Every wait is bounded; on timeout the CTA flags FP_DEV_TIMEOUT, lets issued copies and MMAs
 // finish, frees TMEM and returns.
 // Instances (template flags): kCache -- chunked prefill onto a (paged) K/V cache: each K/V block's
@@ -314,8 +318,9 @@ __device__ __forceinline__ KvIter make_iter(const AttnParams& p, const Unit& u, 
 // ---------------------------------------------------------------------- the kernel -------------
 // kCache: chunked prefill onto a (paged) cache; the plain prefill is compiled separately, with no
 // prefix and direct row indexing. kFp8: e4m3 Q and K (QK^T on kind::f8f6f4), bf16 V.
+// Paired schedule: a unit runs two query tiles of one kv-head (the design above).
 template <int BK, bool kCache, bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
+__device__ __forceinline__ void attn_pairs(const AttnParams& p) {
   using C = Cfg<BK, kFp8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -872,6 +877,556 @@ if (part == 3 && prev_part == 3) {
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ======================================================================= row schedule ============
+// Row schedule (plain bf16 prefill, B = 128), for sparse lists: a unit is one query tile (128 rows of
+// one q-head); both softmax warpgroups split every item's 128 keys (warpgroup 1 keys 0..63, warpgroup
+// 2 keys 64..127, each thread one row of its half) and the two TMEM S buffers alternate between
+// consecutive items, so QK(n+1) runs during softmax(n). Nothing depends on a partner row, so lists of
+// any lengths keep the pipeline full; the price is K/V tiles loaded once per row (no sharing between
+// two rows) and a row-statistics exchange between the two halves per item, which makes it slower
+// than the paired schedule when most blocks are kept (measured at 128K: 23% slower at density 1, 9%
+// at 0.46, 12% faster at 0.06; at 32K 5% faster at 0.32).
+// TMEM: S0 | S1 | O (128 columns each). P of an item overwrites the S columns its own half has read:
+// keys 0..63 packed into columns 0..31, keys 64..127 into columns 96..127.
+namespace rows {
+constexpr int kStages = 2;
+constexpr uint32_t kQBytes = kTileM * kHeadDim * 2, kKBytes = 128 * kHeadDim * 2, kVBytes = kKBytes;
+constexpr uint32_t kSlab = 128 * 128;  // 128 rows x 128 bytes
+constexpr uint32_t kOffQ = 0, kOffK = 2 * kQBytes, kOffV = kOffK + kStages * kKBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
+// q_full[2], q_empty[2], k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2], o_final,
+// pv_done, drain, item[kRing], item_empty[kRing], pair[4] (the two softmax warps of one 32-row
+// quarter exchange row statistics: 64 arrivals per phase, bounded waits), never (test hook)
+constexpr int kNumBars = 4 + 4 * kStages + 4 + 3 + 2 * kRing + 4 + 1;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort, ok
+constexpr uint32_t kOffRing = kOffMisc + 16;
+constexpr uint32_t kOffX = kOffRing + 4 * kRing;               // exchange: float [2 parity][2 half][128], int vote[2][2][4]
+constexpr uint32_t kXBytes = 2 * 2 * 128 * 4 + 2 * 2 * 4 * 4;
+constexpr uint32_t kOffTab = (kOffX + kXBytes + 15) & ~15u;
+constexpr uint32_t smem_bytes(int num_seqs) { return kOffTab + 5 * 4 * (num_seqs + 1) + 8 * (num_seqs + 1) + 16 + 1024; }
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHeadDim, 0, 1);
+}  // namespace rows
+
+__device__ __forceinline__ void attn_rows(const AttnParams& p) {
+  using namespace rows;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV;
+  const uint32_t bar0 = sbase + kOffBar;
+  auto b_q_full = [&](int i) { return bar0 + 8 * i; };
+  auto b_q_empty = [&](int i) { return bar0 + 16 + 8 * i; };
+  auto b_k_full = [&](int i) { return bar0 + 32 + 8 * i; };
+  auto b_k_empty = [&](int i) { return bar0 + 32 + 8 * (kStages + i); };
+  auto b_v_full = [&](int i) { return bar0 + 32 + 8 * (2 * kStages + i); };
+  auto b_v_empty = [&](int i) { return bar0 + 32 + 8 * (3 * kStages + i); };
+  const uint32_t b_s_full0 = bar0 + 32 + 8 * (4 * kStages), b_p_full0 = b_s_full0 + 16;
+  const uint32_t b_o_final = b_p_full0 + 16, b_pv_done = b_o_final + 8, b_drain = b_pv_done + 8;
+  auto b_item = [&](uint32_t x) { return b_drain + 8 + 8 * (x % kRing); };
+  auto b_item_empty = [&](uint32_t x) { return b_drain + 8 + 8 * kRing + 8 * (x % kRing); };
+  auto b_pair = [&](int q) { return b_drain + 8 + 16 * kRing + 8 * q; };
+  const uint32_t b_never = b_drain + 8 + 16 * kRing + 32;
+  volatile int* s_item = reinterpret_cast<volatile int*>(smem + kOffRing);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  int* s_ok = reinterpret_cast<int*>(smem + kOffMisc + 8);
+  volatile float* s_xf = reinterpret_cast<volatile float*>(smem + kOffX);             // [par][half][row]
+  volatile int* s_vote = reinterpret_cast<volatile int*>(smem + kOffX + 2 * 2 * 128 * 4);  // [par][half][q4]
+  const int S = p.seq.num_seqs;
+  int* s_cu = reinterpret_cast<int*>(smem + kOffTab);
+  int* s_cb = s_cu + (S + 1);
+  int* s_ct = s_cb + (S + 1);
+  int* s_pb = s_ct + (S + 1);
+  int* s_ckb = s_pb + (S + 1);
+  long long* s_ib = reinterpret_cast<long long*>(smem + kOffTab + 20 * (S + 1) + 4);
+  s_ib = reinterpret_cast<long long*>(((uintptr_t)s_ib + 7) & ~(uintptr_t)7);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_q_full(i), 1);
+      mbar_init(b_q_empty(i), 1);
+      mbar_init(b_s_full0 + 8 * i, 1);
+      mbar_init(b_p_full0 + 8 * i, 256);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(b_k_full(i), 1);
+      mbar_init(b_k_empty(i), 1);
+      mbar_init(b_v_full(i), 1);
+      mbar_init(b_v_empty(i), 1);
+    }
+    mbar_init(b_o_final, 1);
+    mbar_init(b_pv_done, 1);
+    mbar_init(b_drain, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(b_item(i), 1);
+      mbar_init(b_item_empty(i), kRingReaders);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(b_pair(i), 64);
+    mbar_init(b_never, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), kTmemCols);
+    tmem_relinquish();
+  }
+  // unit table: Hq units (one per q-head) per 128 query rows
+  const bool ok = build_seq_tables(p.seq, s_cu, s_cb, s_ct, s_ib, p.hq, kTileM, p.hq, s_ok, p.dev_status, s_pb, s_ckb) &&
+                  (p.dense || s_ib[S] == p.index_elems);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  if (!ok && threadIdx.x == 0 && !p.dense) dev_flag(p.dev_status, kDevBadProblem);
+  const int num_units = ok ? s_ct[S] : 0;
+  // unit t -> (sequence, kv-head outermost, descending query tile, q-head)
+  auto decode1 = [&](int t, int& s, int& g, int& h, int& qt) {
+    s = find_seq(s_ct, S, t);
+    const int local = t - s_ct[s];
+    const int len = s_cu[s + 1] - s_cu[s];
+    const int ntile = (len + kTileM - 1) / kTileM;
+    const int per_g = ntile * p.group;
+    g = local / per_g;
+    const int rem = local % per_g;
+    qt = ntile - 1 - rem / p.group;
+    h = g * p.group + rem % p.group;
+  };
+  if (wg == 0) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+
+  if (warp == 0) {
+    // =========================================================== producer
+    if (lane == 0) {
+      uint32_t kit = 0, vit = 0, xit = 0;
+      int uc = 0;
+      bool fail = false, bad = false;
+      auto publish = [&](int val) -> bool {
+        if (xit >= (uint32_t)kRing && !mbar_wait(b_item_empty(xit), ((xit / kRing) - 1) & 1, p.wait_limit_ns)) return false;
+        s_item[xit % kRing] = val;
+        mbar_arrive(b_item(xit));
+        ++xit;
+        return true;
+      };
+      int t = blockIdx.x;
+      for (int k = 0;; ++uc) {
+        if (t >= num_units || fail) break;
+        int s, g, h, qt;
+        decode1(t, s, g, h, qt);
+        const int seq0 = s_cu[s], nb = s_cb[s + 1] - s_cb[s];
+        if (!publish(t)) { fail = true; break; }
+        const int qs = uc & 1;
+        if (!mbar_wait(b_q_empty(qs), ((uc >> 1) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+        mbar_arrive_expect_tx(b_q_full(qs), kQBytes);
+        tma_load_2d(sQ + qs * kQBytes, &p.tm_q, b_q_full(qs), h * kHeadDim, seq0 + qt * kTileM);
+        tma_load_2d(sQ + qs * kQBytes + kSlab, &p.tm_q, b_q_full(qs), h * kHeadDim + 64, seq0 + qt * kTileM);
+        // the row's list (B = 128: one query block per tile)
+        const int blk = qt;
+        const int jd = blk;
+        int n = 0;
+        const int32_t* list = nullptr;
+        if (blk < nb) {
+          if (p.dense) n = jd + 1;
+          else {
+            list = p.indices + list_row(s_cb, s_ib, s_pb, s, h, blk);
+            n = min(max(__ldg(p.counts + (long long)h * p.seq.total_blocks + s_cb[s] + blk), 0), jd + 1);
+          }
+        }
+        long long vy = -1;
+        auto load_v = [&](long long y) -> bool {
+          const int vs = vit % kStages;
+          if (!mbar_wait(b_v_empty(vs), ((vit / kStages) & 1) ^ 1, p.wait_limit_ns)) return false;
+          mbar_arrive_expect_tx(b_v_full(vs), kVBytes);
+          tma_load_2d(sV + vs * kVBytes, &p.tm_v, b_v_full(vs), g * kHeadDim, (int32_t)y);
+          tma_load_2d(sV + vs * kVBytes + kSlab, &p.tm_v, b_v_full(vs), g * kHeadDim + 64, (int32_t)y);
+          ++vit;
+          return true;
+        };
+        for (int i = 0; i < n; ++i) {
+          const int j = p.dense ? i : __ldg(list + i);
+          if (j < 0 || j > jd) { bad = true; continue; }
+          const long long y = (long long)seq0 + (long long)j * 128;
+          if (!publish(j)) { fail = true; break; }
+          const int ks = kit % kStages;
+          if (!mbar_wait(b_k_empty(ks), ((kit / kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+          mbar_arrive_expect_tx(b_k_full(ks), kKBytes);
+          tma_load_2d(sK + ks * kKBytes, &p.tm_k, b_k_full(ks), g * kHeadDim, (int32_t)y);
+          tma_load_2d(sK + ks * kKBytes + kSlab, &p.tm_k, b_k_full(ks), g * kHeadDim + 64, (int32_t)y);
+          ++kit;
+          if (vy >= 0 && !load_v(vy)) { fail = true; break; }
+          vy = y;
+          if (*s_abort) { fail = true; break; }
+        }
+        if (!fail && vy >= 0 && !load_v(vy)) fail = true;
+        if (!fail && !publish(kItemEnd)) fail = true;
+        if (!fail) t = next_unit(p.sched, ++k);
+      }
+      if (!fail && !publish(kUnitsEnd)) fail = true;
+      sched_release(p.sched);
+      if (bad) dev_flag(p.dev_status, kDevBadList);
+      if (fail) {
+        *s_abort = 1;
+        dev_flag(p.dev_status, kDevTimeout);
+        for (int i = 0; i < kStages; ++i) {
+          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), ((kit - 1 - i) / kStages) & 1, kDrainLimitNs);
+          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), ((vit - 1 - i) / kStages) & 1, kDrainLimitNs);
+        }
+        for (int i = 0; i < 2 && i < uc + 1; ++i) {
+          const int u_last = uc - i;
+          if (u_last >= 0) mbar_wait(b_q_full(u_last & 1), (u_last >> 1) & 1, kDrainLimitNs);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      uint32_t kit = 0, vit = 0, xit = 0;
+      uint32_t g_it = 0;  // items issued so far (S buffer g_it % 2; phase (g_it / 2) & 1)
+      int uc = 0;
+      bool fail = false;
+      auto read_item = [&](int& e) -> bool {
+        if (!mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns)) return false;
+        e = s_item[xit % kRing];
+        mbar_arrive(b_item_empty(xit));
+        ++xit;
+        return true;
+      };
+      auto qk = [&](uint32_t qbase, uint32_t kbase, uint32_t buf) {
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * kSlab + koff, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * kSlab + koff, 16, 1024);
+          mma_ss(tmem + 128u * buf, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_s_full0 + 8 * buf);
+      };
+      // O += P V of global item gi (P in S buffer gi % 2: keys 0..63 packed in columns 0..31, keys
+      // 64..127 in columns 96..127), V tile vit % kStages
+      auto pv = [&](uint32_t gi, bool first) -> bool {
+        const uint32_t buf = gi & 1;
+        if (!mbar_wait(b_p_full0 + 8 * buf, (gi >> 1) & 1, p.wait_limit_ns)) return false;
+        const int vs = vit % kStages;
+        if (!mbar_wait(b_v_full(vs), (vit / kStages) & 1, p.wait_limit_ns)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sV + vs * kVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kSlab, 1024);
+          const uint32_t acol = 128u * buf + (kk < 4 ? 8u * kk : 96u + 8u * (kk - 4));
+          mma_ts(tmem + 256u, tmem + acol, bdesc, kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(b_pv_done);
+        mma_commit(b_v_empty(vs));
+        ++vit;
+        return true;
+      };
+      for (;; ++uc) {
+        int t;
+        if (!read_item(t)) { fail = true; break; }
+        if (t == kUnitsEnd) break;
+        const int qs = uc & 1;
+        if (!mbar_wait(b_q_full(qs), (uc >> 1) & 1, p.wait_limit_ns)) { fail = true; break; }
+        tc_fence_after();
+        const uint32_t qbase = sQ + qs * kQBytes;
+        int e, n = 0;
+        if (!read_item(e)) { fail = true; break; }
+        while (e != kItemEnd) {
+          const int ks = kit % kStages;
+          if (!mbar_wait(b_k_full(ks), (kit / kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
+          tc_fence_after();
+          qk(qbase, sK + ks * kKBytes, g_it & 1);   // S(n): buffer free since PV(n-2) was issued
+          mma_commit(b_k_empty(ks));
+          ++kit;
+          if (n > 0 && !pv(g_it - 1, n == 1)) { fail = true; break; }  // PV(n-1) once its P is stored
+          ++g_it;
+          ++n;
+          if (!read_item(e)) { fail = true; break; }
+          if (e == kItemEnd) mma_commit(b_q_empty(qs));
+          if (*s_abort) { fail = true; break; }
+        }
+        if (fail) break;
+        if (n > 0) {
+          if (!pv(g_it - 1, n == 1)) { fail = true; break; }
+          mma_commit(b_o_final);
+        } else {
+          mma_commit(b_q_empty(qs));
+        }
+      }
+      if (fail) {
+        *s_abort = 1;
+        dev_flag(p.dev_status, kDevTimeout);
+      }
+      mma_commit(b_drain);
+      mbar_wait(b_drain, 0, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (wg >= 1) {
+    // =========================================================== softmax (one half of every item's keys)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int hf = wg - 1;                    // key half
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t o_col = tmem + lane_off + 256u + 64u * hf;
+    uint32_t g_it = 0;                        // items processed (global, buffer parity)
+    uint32_t xit = 0;
+    int fc = 0;
+    bool fail = false;
+    uint32_t pcnt = 0;  // pair exchanges so far (pair barrier phases)
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(b_pair(q4));
+      const bool okk = !__any_sync(kFull, !mbar_wait(b_pair(q4), pcnt & 1, p.wait_limit_ns));
+      ++pcnt;
+      return okk;
+    };
+    if (p.test_unsignalled_wait && num_units > 0)
+      fail = __any_sync(kFull, !mbar_wait(b_never, 0, p.wait_limit_ns));
+    auto read_entry = [&](int& e) -> bool {
+      if (__any_sync(kFull, !mbar_wait(b_item(xit), (xit / kRing) & 1, p.wait_limit_ns))) return false;
+      e = s_item[xit % kRing];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_item_empty(xit));
+      ++xit;
+      return true;
+    };
+    while (!fail) {
+      int t;
+      if (!read_entry(t)) { fail = true; break; }
+      if (t == kUnitsEnd) break;
+      int s, g, h, qt;
+      decode1(t, s, g, h, qt);
+      const int len = s_cu[s + 1] - s_cu[s];
+      const int qpos = qt * kTileM + r;
+      const bool pad = qpos >= len;
+      float m_run = -INFINITY, l_half = 0.f;
+      int n = 0;
+      while (true) {
+        int e;
+        if (!read_entry(e)) { fail = true; break; }
+        if (e == kItemEnd) break;
+        const int j = e;
+        const uint32_t buf = g_it & 1;
+        const uint32_t par = (g_it >> 1) & 1;
+        if (__any_sync(kFull, !mbar_wait(b_s_full0 + 8 * buf, par, p.wait_limit_ns))) { fail = true; break; }
+        tc_fence_after();
+        const uint32_t s_col = tmem + lane_off + 128u * buf + 64u * hf;
+        const int valid = qpos - j * 128 - 64 * hf;  // my keys 64 hf + c are causal iff c <= valid
+        const bool masked = qpos - j * 128 < 127;    // some key of the block is masked for this row (both halves agree)
+        const float sl2 = p.scale_log2;
+        const uint64_t scale2 = f2_make(sl2, sl2);
+        uint32_t pk[32];
+        bool done = false;
+        if (__all_sync(kFull, pad || (!masked && m_run != -INFINITY))) {
+          const uint64_t negm2 = f2_make(-m_run, -m_run);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+          uint32_t cb[2][32];
+          tmem_ld32(s_col, cb[0]);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_wait_ld();
+            reg_fence32(cb[c & 1]);
+            if (c == 0) tmem_ld32(s_col + 32, cb[1]);
+#pragma unroll
+            for (int e2 = 0; e2 < 32; e2 += 2) {
+              const int pr = 16 * c + e2 / 2;
+              const uint64_t x2 = ffma2(f2_bits(cb[c][e2], cb[c][e2 + 1]), scale2, negm2);
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+              acc[pr & 3] = fadd2(acc[pr & 3], p2);
+              float p0, p1;
+              f2_split(p2, p0, p1);
+              pk[pr] = pack_bf16x2(p0, p1);
+            }
+          }
+          float a0, a1, b0, b1;
+          f2_split(fadd2(acc[0], acc[1]), a0, a1);
+          f2_split(fadd2(acc[2], acc[3]), b0, b1);
+          const float hsum = (a0 + a1) + (b0 + b1);
+          const bool mine = __all_sync(kFull, pad || hsum <= 32768.f);
+          if (lane == 0) s_vote[(g_it & 1) * 8 + hf * 4 + q4] = mine ? 1 : 0;
+          if (!pair_sync()) { fail = true; break; }
+          done = mine && s_vote[(g_it & 1) * 8 + (1 - hf) * 4 + q4] != 0;
+          if (done) l_half += hsum;
+        }
+        if (!done) {
+          uint32_t sr[64];
+          tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const float v0 = (c + 2 * a <= valid) ? __uint_as_float(sr[c + 2 * a]) : -INFINITY;
+              const float v1 = (c + 2 * a + 1 <= valid) ? __uint_as_float(sr[c + 2 * a + 1]) : -INFINITY;
+              sr[c + 2 * a] = __float_as_uint(v0);
+              sr[c + 2 * a + 1] = __float_as_uint(v1);
+              m4[a] = fmax3(m4[a], v0, v1);
+            }
+          }
+          const float hmax = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+          s_xf[(g_it & 1) * 256 + hf * 128 + r] = hmax;
+          if (!pair_sync()) { fail = true; break; }
+          const float mx = fmaxf(hmax, s_xf[(g_it & 1) * 256 + (1 - hf) * 128 + r]);
+          const float m_new = fmaxf(m_run, mx * sl2);
+          const bool grow = m_new > m_run + 8.0f;
+          float alpha = 1.f;
+          if (grow) {
+            alpha = ex2_approx(m_run - m_new);
+            m_run = m_new;
+          }
+          l_half *= alpha;
+          if (n > 0 && __any_sync(kFull, grow)) {
+            // O must hold PV(n-1): S(n) was committed after PV(n-2) only
+            if (__any_sync(kFull, !mbar_wait(b_pv_done, (g_it - 1) & 1, p.wait_limit_ns))) { fail = true; break; }
+            tc_fence_after();
+            const uint64_t a2 = f2_make(alpha, alpha);
+#pragma unroll 1
+            for (int c = 0; c < 64; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(o_col + c, o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int e2 = 0; e2 < 32; e2 += 2) {
+                float lo, hi;
+                f2_split(fmul2(f2_bits(o[e2], o[e2 + 1]), a2), lo, hi);
+                o[e2] = __float_as_uint(lo);
+                o[e2 + 1] = __float_as_uint(hi);
+              }
+              tmem_st32(o_col + c, o);
+            }
+          }
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          const uint64_t negm2 = f2_make(-m_use, -m_use);
+          uint64_t sum2[2] = {0ull, 0ull};
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const uint64_t x2 = ffma2(f2_bits(sr[c], sr[c + 1]), scale2, negm2);
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            const uint64_t p2 = f2_make(ex2_approx(x0), ex2_approx(x1));
+            sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], p2);
+            float p0, p1;
+            f2_split(p2, p0, p1);
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+          float a0, a1, b0, b1;
+          f2_split(sum2[0], a0, a1);
+          f2_split(sum2[1], b0, b1);
+          l_half += (a0 + a1) + (b0 + b1);
+        }
+        tmem_st32(tmem + lane_off + 128u * buf + (hf ? 96u : 0u), pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(b_p_full0 + 8 * buf);
+        ++g_it;
+        ++n;
+      }
+      if (__any_sync(kFull, fail || *s_abort)) { fail = true; break; }
+      const bool row_ok = !pad;
+      const long long row = (long long)s_cu[s] + qpos;
+      // the row's sum: both halves
+      s_xf[(g_it & 1) * 256 + hf * 128 + r] = l_half;
+      if (!pair_sync()) { fail = true; break; }
+      const float l_run = l_half + s_xf[(g_it & 1) * 256 + (1 - hf) * 128 + r];
+      if (!pair_sync()) { fail = true; break; }  // both read before the exchange area is reused
+      if (n == 0) {
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (row * p.hq + h) * kHeadDim + 64 * hf);
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          if (p.lse && hf == 0) p.lse[(long long)h * p.seq.total_tokens + row] = -INFINITY;
+        }
+        continue;
+      }
+      if (__any_sync(kFull, !mbar_wait(b_o_final, fc & 1, p.wait_limit_ns))) { fail = true; break; }
+      ++fc;
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      uint16_t* orow = p.out + (row * p.hq + h) * kHeadDim + 64 * hf;
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(o_col + c, o);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2)
+          w[e2] = pack_bf16x2(__uint_as_float(o[2 * e2]) * inv_l, __uint_as_float(o[2 * e2 + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
+          dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+        }
+      }
+      if (row_ok && p.lse && hf == 0) {
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        p.lse[(long long)h * p.seq.total_tokens + row] =
+            l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+      }
+      tc_fence_before();
+    }
+    if (fail) {
+      *s_abort = 1;
+      dev_flag(p.dev_status, kDevTimeout);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Schedule choice (plain bf16 prefill, B = 128): the row schedule when fewer than 40% of the causal
+// blocks are kept. Every CTA of both kernels sums the list counts (4 bytes per list) before it starts,
+// so both take the same decision; p.units forces either schedule. Call with every thread of the CTA.
+__device__ __forceinline__ bool rows_chosen(const AttnParams& p) {
+  if (p.units != 0) return p.units == 2;
+  if (p.dense || p.index_elems <= 0) return false;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned long long* s_kept = reinterpret_cast<unsigned long long*>(smem_raw);  // scratch before set-up
+  if (threadIdx.x == 0) *s_kept = 0ull;
+  __syncthreads();
+  const long long n = (long long)p.hq * p.seq.total_blocks;
+  unsigned long long part = 0ull;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) part += (unsigned)max(__ldg(p.counts + i), 0);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(kFull, part, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(s_kept, part);
+  __syncthreads();
+  const bool rows = 5ull * *s_kept < 2ull * (unsigned long long)p.index_elems;
+  __syncthreads();  // the scratch word is part of the set-up area of either schedule
+  return rows;
+}
+
+// The paired schedule (every instance); the plain bf16 B = 128 instance returns at once when the row
+// schedule is chosen, and attn_rows_kernel, launched right after it, runs the lists instead (two
+// kernels, so that each schedule keeps its own code and register allocation).
+template <int BK, bool kCache, bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
+  if constexpr (BK == 128 && !kCache && !kFp8)
+    if (rows_chosen(p)) return;
+  attn_pairs<BK, kCache, kFp8>(p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_rows_kernel(const __grid_constant__ AttnParams p) {
+  if (!rows_chosen(p)) return;
+  attn_rows(p);
+}
+
 template <int BK, bool kCache, bool kFp8>
 static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
   static unsigned long long attr_done[kMaxCachedDevices] = {};
@@ -879,7 +1434,19 @@ static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st)
                                attr_done);
   if (e != cudaSuccess) return e;
   attn_kernel<BK, kCache, kFp8><<<grid, kThreads, Cfg<BK, kFp8>::smem_bytes(p.seq.num_seqs), st>>>(p);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if constexpr (BK == 128 && !kCache && !kFp8) {
+    if (!p.dense && p.units != 1) {  // the row schedule's kernel (returns at once unless chosen)
+      static_assert(rows::smem_bytes(kMaxSeqs) <= 227 * 1024, "shared memory per CTA");
+      static unsigned long long attr_rows[kMaxCachedDevices] = {};
+      if ((e = set_max_smem(reinterpret_cast<const void*>(attn_rows_kernel), rows::smem_bytes(kMaxSeqs), attr_rows)) !=
+          cudaSuccess)
+        return e;
+      attn_rows_kernel<<<grid, kThreads, rows::smem_bytes(p.seq.num_seqs), st>>>(p);
+      e = cudaGetLastError();
+    }
+  }
+  return e;
 }
 
 cudaError_t launch_attn(const AttnParams& p, int grid, cudaStream_t st) {

@@ -102,6 +102,7 @@ struct __align__(64) AttnParams {
   int32_t* dev_status;
   uint64_t wait_limit_ns;
   int32_t test_unsignalled_wait;  // test hook: softmax warps first wait on a barrier nothing signals
+  int32_t units;                  // attention schedule: 0 by list density, 1 tile pairs, 2 single tiles
   int32_t fp8;                    // 1: tm_q / tm_k are e4m3 (uint8) maps, box {128, rows}; scales folded into scale_log2
   int32_t* sched;                 // work counter (next unit, finished CTAs), zero at launch and exit; or null
   const int8_t* q_exp;            // fp8 with per-block scales: q-block scale 2^q_exp[global block * hq + h], or null

@@ -15,8 +15,10 @@ def _cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
-def test_wait_that_nothing_signals_times_out_and_context_survives(monkeypatch):
+@pytest.mark.parametrize("units", ["pairs", "rows"])
+def test_wait_that_nothing_signals_times_out_and_context_survives(monkeypatch, units):
     import block_sparse_long_causal_b200 as fp
+    monkeypatch.setenv("FP_ATTN_UNITS", units)  # both attention schedules
     x = synth.random_inputs((700, 300), 4, 2, 128, seed=41)
     good = gpu_prefill(x, 4, 2, 128, 0.0)
     monkeypatch.setenv("FP_TEST_UNSIGNALLED_WAIT", "1")

@@ -5,7 +5,9 @@ order differs for each). Logits that jump half-way along the key axis make the r
 by more than the lazy-rescale margin inside those runs, so O is rescaled between items of a run.
 
 The lists are valid method outputs in form (ascending, sink and diagonal present) but are chosen
-here, not by the search; the oracle attends exactly the same blocks.
+here, not by the search; the oracle attends exactly the same blocks. Each case runs under both
+attention schedules (FP_ATTN_UNITS): tile pairs, and single tiles whose two softmax warpgroups split
+every item's keys (plain B = 128; with B = 64 both runs take the pairs).
 """
 import numpy as np
 import pytest
@@ -40,9 +42,11 @@ def _lists(nb, hq, B, dens_odd, dens_even, rng):
     (2944, 6, 2, 128, 0.7, 0.2, 0.0),     # G = 3, odd tile count: one-slot units run alone
     (2048, 4, 2, 64, 0.8, 0.15, 47.0),    # B = 64: two lists per slot
 ])
-def test_attention_on_item_patterns(L, hq, hkv, B, dens_odd, dens_even, step):
+@pytest.mark.parametrize("units", ["pairs", "rows"])
+def test_attention_on_item_patterns(L, hq, hkv, B, dens_odd, dens_even, step, units, monkeypatch):
     import torch
     import block_sparse_long_causal_b200 as fp
+    monkeypatch.setenv("FP_ATTN_UNITS", units)  # rows: the single-tile schedule (B = 128 only)
     rng = np.random.default_rng(L + 7 * hq + B)
     x = synth.random_inputs((L,), hq, hkv, 128, seed=L + hq, scale=1.0)
     if step:

@@ -32,9 +32,10 @@ def _attn(p, q, k, v, counts, indices, dense):
     return bf16_to_np(out), lse.cpu().numpy()
 
 
-@pytest.mark.parametrize("B", [64, 128])
-def test_counter_and_fixed_schedule_agree_bit_for_bit(B):
+@pytest.mark.parametrize("B,units", [(64, "pairs"), (128, "pairs"), (128, "rows")])
+def test_counter_and_fixed_schedule_agree_bit_for_bit(B, units, monkeypatch):
     import block_sparse_long_causal_b200 as fp
+    monkeypatch.setenv("FP_ATTN_UNITS", units)
     # three sequences of uneven length and a selective threshold: lists of very different lengths
     x = synth.random_inputs((3000, 700, 5100), 8, 2, 128, seed=61, scale=2.0)
     cu = x["cu_seqlens"]
@@ -101,9 +102,11 @@ def test_counter_in_a_cuda_graph_replays():
     del g
 
 
-def test_counter_is_zero_after_a_launch_whose_waits_ran_out(monkeypatch):
+@pytest.mark.parametrize("units", ["pairs", "rows"])
+def test_counter_is_zero_after_a_launch_whose_waits_ran_out(monkeypatch, units):
     import torch
     import block_sparse_long_causal_b200 as fp
+    monkeypatch.setenv("FP_ATTN_UNITS", units)
     x = synth.random_inputs((900, 300), 4, 2, 128, seed=64)
     p = fp.problem(x["cu_seqlens"], 4, 2, 128, 128)
     q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
