@@ -502,32 +502,31 @@ __device__ __forceinline__ void attn_pairs(const AttnParams& p) {
         const int vs = vit % C::kStages;
         if (!mbar_wait(b_v_full(vs), (vit / C::kStages) & 1, p.wait_limit_ns)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + vs * C::kVBytes;
+        const uint64_t vdesc = sdesc_sw128(sV + vs * C::kVBytes, C::kSlabKV, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSlabKV, 1024);
-          mma_ts(tmem + tmem_o(k), tmem + tmem_s(k) + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)  // 16 keys = 16 rows of 128 bytes per step
+          mma_ts(tmem + tmem_o(k), tmem + tmem_s(k) + kk * 8, desc_advance(vdesc, kk * (2048 >> 4)), C::kIdescPV,
+                 (!first || kk > 0) ? 1u : 0u);
         return true;
       };
       // S_k = Q_k K^T for the current item (K tile at kbase)
       auto qk = [&](int k, uint32_t kbase) {
-        const uint32_t qbase = sQ + k * C::kQBytes;
+        const uint64_t qdesc = sdesc_sw128(sQ + k * C::kQBytes, 16, 1024);
+        const uint64_t kdesc = sdesc_sw128(kbase, 16, 1024);
         if constexpr (kFp8) {
           // 4 steps of 32 e4m3 = 32 bytes inside the single 128-byte swizzle atom
 #pragma unroll
-          for (int kk = 0; kk < kHeadDim / 32; ++kk) {
-            const uint64_t adesc = sdesc_sw128(qbase + kk * 32, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(kbase + kk * 32, 16, 1024);
-            mma_ss_f8(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kHeadDim / 32; ++kk)
+            mma_ss_f8(tmem + tmem_s(k), desc_advance(qdesc, kk * 2), desc_advance(kdesc, kk * 2), C::kIdescQK,
+                      kk > 0 ? 1u : 0u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
-            const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * C::kSlabQ + koff, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * C::kSlabK + koff, 16, 1024);
-            mma_ss(tmem + tmem_s(k), adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+            // 16 bf16 = 32 bytes inside the swizzle atom; 64 columns per slab
+            const uint32_t qoff = ((kk >> 2) * C::kSlabQ + (kk & 3) * 32) >> 4;
+            const uint32_t koff = ((kk >> 2) * C::kSlabK + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + tmem_s(k), desc_advance(qdesc, qoff), desc_advance(kdesc, koff), C::kIdescQK,
+                   kk > 0 ? 1u : 0u);
           }
         }
         mma_commit(b_s_full0 + 8 * k);
@@ -883,24 +882,26 @@ if (part == 3 && prev_part == 3) {
 // 2 keys 64..127, each thread one row of its half) and the two TMEM S buffers alternate between
 // consecutive items, so QK(n+1) runs during softmax(n). Nothing depends on a partner row, so lists of
 // any lengths keep the pipeline full; the price is K/V tiles loaded once per row (no sharing between
-// two rows) and a row-statistics exchange between the two halves per item, which makes it slower
-// than the paired schedule when most blocks are kept (measured at 128K: 23% slower at density 1, 9%
-// at 0.46, 12% faster at 0.06; at 32K 5% faster at 0.32).
-// TMEM: S0 | S1 | O (128 columns each). P of an item overwrites the S columns its own half has read:
-// keys 0..63 packed into columns 0..31, keys 64..127 into columns 96..127.
+// two rows), which makes it slower than the paired schedule when most blocks are kept (measured at
+// 128K: 23% slower at density 1, 9% at 0.46, 12% faster at 0.06; at 32K 5% faster at 0.32).
+// Each half keeps its own running max, row sum and accumulator (O0 = P0 V[0, 64), O1 = P1 V[64,
+// 128)), so the halves never wait for each other inside a unit; the epilogue exchanges (max, sum)
+// once and writes (a0 O0 + a1 O1) / (a0 l0 + a1 l1) with a_h = 2^(m_h - max(m0, m1)).
+// TMEM: S0 | S1 | O0 | O1 (128 columns each). P of an item overwrites the S columns its own half
+// has read: keys 0..63 packed into columns 0..31, keys 64..127 into columns 96..127.
 namespace rows {
-constexpr int kStages = 2;
+constexpr int kQBufs = 2, kKStages = 2, kVStages = 2;  // Q tiles, K ring, V ring
 constexpr uint32_t kQBytes = kTileM * kHeadDim * 2, kKBytes = 128 * kHeadDim * 2, kVBytes = kKBytes;
 constexpr uint32_t kSlab = 128 * 128;  // 128 rows x 128 bytes
-constexpr uint32_t kOffQ = 0, kOffK = 2 * kQBytes, kOffV = kOffK + kStages * kKBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
+constexpr uint32_t kOffQ = 0, kOffK = kQBufs * kQBytes, kOffV = kOffK + kKStages * kKBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kVBytes;
 // q_full[2], q_empty[2], k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2], o_final,
 // pv_done, drain, item[kRing], item_empty[kRing], pair[4] (the two softmax warps of one 32-row
 // quarter exchange row statistics: 64 arrivals per phase, bounded waits), never (test hook)
-constexpr int kNumBars = 4 + 4 * kStages + 4 + 3 + 2 * kRing + 4 + 1;
+constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 4 + 3 + 2 * kRing + 4 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort, ok
 constexpr uint32_t kOffRing = kOffMisc + 16;
-constexpr uint32_t kOffX = kOffRing + 4 * kRing;               // exchange: float [2 parity][2 half][128], int vote[2][2][4]
+constexpr uint32_t kOffX = kOffRing + 4 * kRing;               // exchange: float max[2 half][128], sum[2 half][128]
 constexpr uint32_t kXBytes = 2 * 2 * 128 * 4 + 2 * 2 * 4 * 4;
 constexpr uint32_t kOffTab = (kOffX + kXBytes + 15) & ~15u;
 constexpr uint32_t smem_bytes(int num_seqs) { return kOffTab + 5 * 4 * (num_seqs + 1) + 8 * (num_seqs + 1) + 16 + 1024; }
@@ -918,10 +919,10 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
   auto b_q_full = [&](int i) { return bar0 + 8 * i; };
   auto b_q_empty = [&](int i) { return bar0 + 16 + 8 * i; };
   auto b_k_full = [&](int i) { return bar0 + 32 + 8 * i; };
-  auto b_k_empty = [&](int i) { return bar0 + 32 + 8 * (kStages + i); };
-  auto b_v_full = [&](int i) { return bar0 + 32 + 8 * (2 * kStages + i); };
-  auto b_v_empty = [&](int i) { return bar0 + 32 + 8 * (3 * kStages + i); };
-  const uint32_t b_s_full0 = bar0 + 32 + 8 * (4 * kStages), b_p_full0 = b_s_full0 + 16;
+  auto b_k_empty = [&](int i) { return bar0 + 32 + 8 * (kKStages + i); };
+  auto b_v_full = [&](int i) { return bar0 + 32 + 8 * (2 * kKStages + i); };
+  auto b_v_empty = [&](int i) { return bar0 + 32 + 8 * (2 * kKStages + kVStages + i); };
+  const uint32_t b_s_full0 = bar0 + 32 + 8 * (2 * kKStages + 2 * kVStages), b_p_full0 = b_s_full0 + 16;
   const uint32_t b_o_final = b_p_full0 + 16, b_pv_done = b_o_final + 8, b_drain = b_pv_done + 8;
   auto b_item = [&](uint32_t x) { return b_drain + 8 + 8 * (x % kRing); };
   auto b_item_empty = [&](uint32_t x) { return b_drain + 8 + 8 * kRing + 8 * (x % kRing); };
@@ -932,7 +933,6 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* s_ok = reinterpret_cast<int*>(smem + kOffMisc + 8);
   volatile float* s_xf = reinterpret_cast<volatile float*>(smem + kOffX);             // [par][half][row]
-  volatile int* s_vote = reinterpret_cast<volatile int*>(smem + kOffX + 2 * 2 * 128 * 4);  // [par][half][q4]
   const int S = p.seq.num_seqs;
   int* s_cu = reinterpret_cast<int*>(smem + kOffTab);
   int* s_cb = s_cu + (S + 1);
@@ -950,9 +950,11 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
       mbar_init(b_s_full0 + 8 * i, 1);
       mbar_init(b_p_full0 + 8 * i, 256);
     }
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(b_k_full(i), 1);
       mbar_init(b_k_empty(i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(b_v_full(i), 1);
       mbar_init(b_v_empty(i), 1);
     }
@@ -1020,8 +1022,8 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
         decode1(t, s, g, h, qt);
         const int seq0 = s_cu[s], nb = s_cb[s + 1] - s_cb[s];
         if (!publish(t)) { fail = true; break; }
-        const int qs = uc & 1;
-        if (!mbar_wait(b_q_empty(qs), ((uc >> 1) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+        const int qs = uc % kQBufs;
+        if (!mbar_wait(b_q_empty(qs), ((uc / kQBufs) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
         mbar_arrive_expect_tx(b_q_full(qs), kQBytes);
         tma_load_2d(sQ + qs * kQBytes, &p.tm_q, b_q_full(qs), h * kHeadDim, seq0 + qt * kTileM);
         tma_load_2d(sQ + qs * kQBytes + kSlab, &p.tm_q, b_q_full(qs), h * kHeadDim + 64, seq0 + qt * kTileM);
@@ -1039,8 +1041,8 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
         }
         long long vy = -1;
         auto load_v = [&](long long y) -> bool {
-          const int vs = vit % kStages;
-          if (!mbar_wait(b_v_empty(vs), ((vit / kStages) & 1) ^ 1, p.wait_limit_ns)) return false;
+          const int vs = vit % kVStages;
+          if (!mbar_wait(b_v_empty(vs), ((vit / kVStages) & 1) ^ 1, p.wait_limit_ns)) return false;
           mbar_arrive_expect_tx(b_v_full(vs), kVBytes);
           tma_load_2d(sV + vs * kVBytes, &p.tm_v, b_v_full(vs), g * kHeadDim, (int32_t)y);
           tma_load_2d(sV + vs * kVBytes + kSlab, &p.tm_v, b_v_full(vs), g * kHeadDim + 64, (int32_t)y);
@@ -1052,8 +1054,8 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           if (j < 0 || j > jd) { bad = true; continue; }
           const long long y = (long long)seq0 + (long long)j * 128;
           if (!publish(j)) { fail = true; break; }
-          const int ks = kit % kStages;
-          if (!mbar_wait(b_k_empty(ks), ((kit / kStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+          const int ks = kit % kKStages;
+          if (!mbar_wait(b_k_empty(ks), ((kit / kKStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
           mbar_arrive_expect_tx(b_k_full(ks), kKBytes);
           tma_load_2d(sK + ks * kKBytes, &p.tm_k, b_k_full(ks), g * kHeadDim, (int32_t)y);
           tma_load_2d(sK + ks * kKBytes + kSlab, &p.tm_k, b_k_full(ks), g * kHeadDim + 64, (int32_t)y);
@@ -1072,13 +1074,13 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
       if (fail) {
         *s_abort = 1;
         dev_flag(p.dev_status, kDevTimeout);
-        for (int i = 0; i < kStages; ++i) {
-          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), ((kit - 1 - i) / kStages) & 1, kDrainLimitNs);
-          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), ((vit - 1 - i) / kStages) & 1, kDrainLimitNs);
-        }
-        for (int i = 0; i < 2 && i < uc + 1; ++i) {
+        for (int i = 0; i < kKStages; ++i)
+          if (kit > (uint32_t)i) mbar_wait(b_k_full(i), ((kit - 1 - i) / kKStages) & 1, kDrainLimitNs);
+        for (int i = 0; i < kVStages; ++i)
+          if (vit > (uint32_t)i) mbar_wait(b_v_full(i), ((vit - 1 - i) / kVStages) & 1, kDrainLimitNs);
+        for (int i = 0; i < kQBufs && i < uc + 1; ++i) {
           const int u_last = uc - i;
-          if (u_last >= 0) mbar_wait(b_q_full(u_last & 1), (u_last >> 1) & 1, kDrainLimitNs);
+          if (u_last >= 0) mbar_wait(b_q_full(u_last % kQBufs), (u_last / kQBufs) & 1, kDrainLimitNs);
         }
       }
     }
@@ -1098,29 +1100,28 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
         return true;
       };
       auto qk = [&](uint32_t qbase, uint32_t kbase, uint32_t buf) {
+        const uint64_t qdesc = sdesc_sw128(qbase, 16, 1024), kdesc = sdesc_sw128(kbase, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(qbase + (kk >> 2) * kSlab + koff, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(kbase + (kk >> 2) * kSlab + koff, 16, 1024);
-          mma_ss(tmem + 128u * buf, adesc, bdesc, kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kSlab + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + 128u * buf, desc_advance(qdesc, off), desc_advance(kdesc, off), kIdescQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(b_s_full0 + 8 * buf);
       };
-      // O += P V of global item gi (P in S buffer gi % 2: keys 0..63 packed in columns 0..31, keys
-      // 64..127 in columns 96..127), V tile vit % kStages
+      // O0 += P0 V[0, 64) and O1 += P1 V[64, 128) of global item gi (P in S buffer gi % 2: keys
+      // 0..63 packed in columns 0..31, keys 64..127 in columns 96..127), V tile vit % kVStages
       auto pv = [&](uint32_t gi, bool first) -> bool {
         const uint32_t buf = gi & 1;
         if (!mbar_wait(b_p_full0 + 8 * buf, (gi >> 1) & 1, p.wait_limit_ns)) return false;
-        const int vs = vit % kStages;
-        if (!mbar_wait(b_v_full(vs), (vit / kStages) & 1, p.wait_limit_ns)) return false;
+        const int vs = vit % kVStages;
+        if (!mbar_wait(b_v_full(vs), (vit / kVStages) & 1, p.wait_limit_ns)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + vs * kVBytes;
+        const uint64_t vdesc = sdesc_sw128(sV + vs * kVBytes, kSlab, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kSlab, 1024);
+          const uint64_t bdesc = desc_advance(vdesc, kk * (2048 >> 4));
           const uint32_t acol = 128u * buf + (kk < 4 ? 8u * kk : 96u + 8u * (kk - 4));
-          mma_ts(tmem + 256u, tmem + acol, bdesc, kIdescPV, (!first || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + (kk < 4 ? 256u : 384u), tmem + acol, bdesc, kIdescPV, (!first || (kk & 3) > 0) ? 1u : 0u);
         }
         mma_commit(b_pv_done);
         mma_commit(b_v_empty(vs));
@@ -1131,15 +1132,15 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
         int t;
         if (!read_item(t)) { fail = true; break; }
         if (t == kUnitsEnd) break;
-        const int qs = uc & 1;
-        if (!mbar_wait(b_q_full(qs), (uc >> 1) & 1, p.wait_limit_ns)) { fail = true; break; }
+        const int qs = uc % kQBufs;
+        if (!mbar_wait(b_q_full(qs), (uc / kQBufs) & 1, p.wait_limit_ns)) { fail = true; break; }
         tc_fence_after();
         const uint32_t qbase = sQ + qs * kQBytes;
         int e, n = 0;
         if (!read_item(e)) { fail = true; break; }
         while (e != kItemEnd) {
-          const int ks = kit % kStages;
-          if (!mbar_wait(b_k_full(ks), (kit / kStages) & 1, p.wait_limit_ns)) { fail = true; break; }
+          const int ks = kit % kKStages;
+          if (!mbar_wait(b_k_full(ks), (kit / kKStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
           qk(qbase, sK + ks * kKBytes, g_it & 1);   // S(n): buffer free since PV(n-2) was issued
           mma_commit(b_k_empty(ks));
@@ -1174,7 +1175,7 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t o_col = tmem + lane_off + 256u + 64u * hf;
+    const uint32_t o_col = tmem + lane_off + 256u + 128u * hf;  // this half's own O (all 128 columns)
     uint32_t g_it = 0;                        // items processed (global, buffer parity)
     uint32_t xit = 0;
     int fc = 0;
@@ -1218,7 +1219,7 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
         tc_fence_after();
         const uint32_t s_col = tmem + lane_off + 128u * buf + 64u * hf;
         const int valid = qpos - j * 128 - 64 * hf;  // my keys 64 hf + c are causal iff c <= valid
-        const bool masked = qpos - j * 128 < 127;    // some key of the block is masked for this row (both halves agree)
+        const bool masked = valid < 63;              // some key of my half is masked for this row
         const float sl2 = p.scale_log2;
         const uint64_t scale2 = f2_make(sl2, sl2);
         uint32_t pk[32];
@@ -1250,10 +1251,7 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           f2_split(fadd2(acc[0], acc[1]), a0, a1);
           f2_split(fadd2(acc[2], acc[3]), b0, b1);
           const float hsum = (a0 + a1) + (b0 + b1);
-          const bool mine = __all_sync(kFull, pad || hsum <= 32768.f);
-          if (lane == 0) s_vote[(g_it & 1) * 8 + hf * 4 + q4] = mine ? 1 : 0;
-          if (!pair_sync()) { fail = true; break; }
-          done = mine && s_vote[(g_it & 1) * 8 + (1 - hf) * 4 + q4] != 0;
+          done = __all_sync(kFull, pad || hsum <= 32768.f);
           if (done) l_half += hsum;
         }
         if (!done) {
@@ -1276,10 +1274,7 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
             }
           }
           const float hmax = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-          s_xf[(g_it & 1) * 256 + hf * 128 + r] = hmax;
-          if (!pair_sync()) { fail = true; break; }
-          const float mx = fmaxf(hmax, s_xf[(g_it & 1) * 256 + (1 - hf) * 128 + r]);
-          const float m_new = fmaxf(m_run, mx * sl2);
+          const float m_new = fmaxf(m_run, hmax * sl2);
           const bool grow = m_new > m_run + 8.0f;
           float alpha = 1.f;
           if (grow) {
@@ -1293,7 +1288,7 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
             tc_fence_after();
             const uint64_t a2 = f2_make(alpha, alpha);
 #pragma unroll 1
-            for (int c = 0; c < 64; c += 32) {
+            for (int c = 0; c < 128; c += 32) {
               uint32_t o[32];
               tmem_ld32(o_col + c, o);
               tmem_wait_ld();
@@ -1337,11 +1332,16 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
       if (__any_sync(kFull, fail || *s_abort)) { fail = true; break; }
       const bool row_ok = !pad;
       const long long row = (long long)s_cu[s] + qpos;
-      // the row's sum: both halves
-      s_xf[(g_it & 1) * 256 + hf * 128 + r] = l_half;
+      // the row's statistics: each half's running max and sum (both relative to its own max)
+      s_xf[hf * 128 + r] = m_run;
+      s_xf[256 + hf * 128 + r] = l_half;
       if (!pair_sync()) { fail = true; break; }
-      const float l_run = l_half + s_xf[(g_it & 1) * 256 + (1 - hf) * 128 + r];
+      const float m_oth = s_xf[(1 - hf) * 128 + r], l_oth = s_xf[256 + (1 - hf) * 128 + r];
       if (!pair_sync()) { fail = true; break; }  // both read before the exchange area is reused
+      const float m_row = fmaxf(m_run, m_oth);
+      const float m_use = (m_row == -INFINITY) ? 0.f : m_row;
+      const float a_me = ex2_approx(m_run - m_use), a_oth = ex2_approx(m_oth - m_use);  // 0 for an empty half
+      const float l_run = l_half * a_me + l_oth * a_oth;
       if (n == 0) {
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (row * p.hq + h) * kHeadDim + 64 * hf);
@@ -1354,16 +1354,21 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
       ++fc;
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      // output columns 64 hf .. 64 hf + 63: O0 and O1 there, each weighted by its half's factor
+      const float w0 = (hf == 0 ? a_me : a_oth) * inv_l, w1 = (hf == 0 ? a_oth : a_me) * inv_l;
+      const uint32_t o0_col = tmem + lane_off + 256u + 64u * hf;
       uint16_t* orow = p.out + (row * p.hq + h) * kHeadDim + 64 * hf;
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(o_col + c, o);
+        uint32_t o[32], o1[32];
+        tmem_ld32(o0_col + c, o);
+        tmem_ld32(o0_col + 128u + c, o1);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2)
-          w[e2] = pack_bf16x2(__uint_as_float(o[2 * e2]) * inv_l, __uint_as_float(o[2 * e2 + 1]) * inv_l);
+          w[e2] = pack_bf16x2(fmaf(__uint_as_float(o[2 * e2]), w0, __uint_as_float(o1[2 * e2]) * w1),
+                              fmaf(__uint_as_float(o[2 * e2 + 1]), w0, __uint_as_float(o1[2 * e2 + 1]) * w1));
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -1372,11 +1377,9 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
         }
       }
-      if (row_ok && p.lse && hf == 0) {
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      if (row_ok && p.lse && hf == 0)
         p.lse[(long long)h * p.seq.total_tokens + row] =
             l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
-      }
       tc_fence_before();
     }
     if (fail) {

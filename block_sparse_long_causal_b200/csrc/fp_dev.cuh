@@ -179,6 +179,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
+// The same descriptor for an operand `off16` 16-byte units further on: one 32-bit add on the start
+// address field. Every operand tile lies below 256 KB of the shared window, so the field does not
+// overflow into the leading byte offset (the MMA issue loops build one descriptor per tile and
+// advance it per K step, which keeps the issuing thread's instruction count down).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t off16) {
+  return (d & 0xFFFFFFFF00000000ull) | (uint64_t)((uint32_t)d + off16);
+}
 
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 accumulate, dense:
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
