@@ -895,10 +895,15 @@ constexpr uint32_t kQBytes = kTileM * kHeadDim * 2, kKBytes = 128 * kHeadDim * 2
 constexpr uint32_t kSlab = 128 * 128;  // 128 rows x 128 bytes
 constexpr uint32_t kOffQ = 0, kOffK = kQBufs * kQBytes, kOffV = kOffK + kKStages * kKBytes;
 constexpr uint32_t kOffBar = kOffV + kVStages * kVBytes;
-// q_full[2], q_empty[2], k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2], o_final,
-// pv_done, drain, item[kRing], item_empty[kRing], pair[4] (the two softmax warps of one 32-row
-// quarter exchange row statistics: 64 arrivals per phase, bounded waits), never (test hook)
-constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 4 + 3 + 2 * kRing + 4 + 1;
+// q_full[2], q_empty[2], k_full[], v_full[], v_empty[], s_full[2], p_full[2], o_final, drain,
+// item[kRing], item_empty[kRing], pair[4] (the two softmax warps of one 32-row quarter exchange row
+// statistics: 64 arrivals per phase, bounded waits), never (test hook).
+// A K stage is released by the S barrier of the QK that read it (K stage n % 2 = S buffer n % 2),
+// and an O rescale waits for the previous item's PV on that PV's V-empty barrier: two commits per
+// item fewer for the issuing thread. Neither wait can alias a later phase: the next phase of either
+// barrier needs a tile or a P that the waiter has not produced yet.
+static_assert(kKStages == 2, "K stages are released through the two S buffers' barriers");
+constexpr int kNumBars = 4 + kKStages + 2 * kVStages + 4 + 2 + 2 * kRing + 4 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort, ok
 constexpr uint32_t kOffRing = kOffMisc + 16;
 constexpr uint32_t kOffX = kOffRing + 4 * kRing;               // exchange: float max[2 half][128], sum[2 half][128]
@@ -919,11 +924,10 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
   auto b_q_full = [&](int i) { return bar0 + 8 * i; };
   auto b_q_empty = [&](int i) { return bar0 + 16 + 8 * i; };
   auto b_k_full = [&](int i) { return bar0 + 32 + 8 * i; };
-  auto b_k_empty = [&](int i) { return bar0 + 32 + 8 * (kKStages + i); };
-  auto b_v_full = [&](int i) { return bar0 + 32 + 8 * (2 * kKStages + i); };
-  auto b_v_empty = [&](int i) { return bar0 + 32 + 8 * (2 * kKStages + kVStages + i); };
-  const uint32_t b_s_full0 = bar0 + 32 + 8 * (2 * kKStages + 2 * kVStages), b_p_full0 = b_s_full0 + 16;
-  const uint32_t b_o_final = b_p_full0 + 16, b_pv_done = b_o_final + 8, b_drain = b_pv_done + 8;
+  auto b_v_full = [&](int i) { return bar0 + 32 + 8 * (kKStages + i); };
+  auto b_v_empty = [&](int i) { return bar0 + 32 + 8 * (kKStages + kVStages + i); };
+  const uint32_t b_s_full0 = bar0 + 32 + 8 * (kKStages + 2 * kVStages), b_p_full0 = b_s_full0 + 16;
+  const uint32_t b_o_final = b_p_full0 + 16, b_drain = b_o_final + 8;
   auto b_item = [&](uint32_t x) { return b_drain + 8 + 8 * (x % kRing); };
   auto b_item_empty = [&](uint32_t x) { return b_drain + 8 + 8 * kRing + 8 * (x % kRing); };
   auto b_pair = [&](int q) { return b_drain + 8 + 16 * kRing + 8 * q; };
@@ -950,16 +954,12 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
       mbar_init(b_s_full0 + 8 * i, 1);
       mbar_init(b_p_full0 + 8 * i, 256);
     }
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(b_k_full(i), 1);
-      mbar_init(b_k_empty(i), 1);
-    }
+    for (int i = 0; i < kKStages; ++i) mbar_init(b_k_full(i), 1);
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(b_v_full(i), 1);
       mbar_init(b_v_empty(i), 1);
     }
     mbar_init(b_o_final, 1);
-    mbar_init(b_pv_done, 1);
     mbar_init(b_drain, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(b_item(i), 1);
@@ -1055,7 +1055,9 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           const long long y = (long long)seq0 + (long long)j * 128;
           if (!publish(j)) { fail = true; break; }
           const int ks = kit % kKStages;
-          if (!mbar_wait(b_k_empty(ks), ((kit / kKStages) & 1) ^ 1, p.wait_limit_ns)) { fail = true; break; }
+          // stage ks is free once QK(kit - 2), which read it, is done (S buffer ks, that QK's phase)
+          if (kit >= (uint32_t)kKStages &&
+              !mbar_wait(b_s_full0 + 8 * ks, ((kit - kKStages) / 2) & 1, p.wait_limit_ns)) { fail = true; break; }
           mbar_arrive_expect_tx(b_k_full(ks), kKBytes);
           tma_load_2d(sK + ks * kKBytes, &p.tm_k, b_k_full(ks), g * kHeadDim, (int32_t)y);
           tma_load_2d(sK + ks * kKBytes + kSlab, &p.tm_k, b_k_full(ks), g * kHeadDim + 64, (int32_t)y);
@@ -1123,7 +1125,6 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           const uint32_t acol = 128u * buf + (kk < 4 ? 8u * kk : 96u + 8u * (kk - 4));
           mma_ts(tmem + (kk < 4 ? 256u : 384u), tmem + acol, bdesc, kIdescPV, (!first || (kk & 3) > 0) ? 1u : 0u);
         }
-        mma_commit(b_pv_done);
         mma_commit(b_v_empty(vs));
         ++vit;
         return true;
@@ -1143,7 +1144,6 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           if (!mbar_wait(b_k_full(ks), (kit / kKStages) & 1, p.wait_limit_ns)) { fail = true; break; }
           tc_fence_after();
           qk(qbase, sK + ks * kKBytes, g_it & 1);   // S(n): buffer free since PV(n-2) was issued
-          mma_commit(b_k_empty(ks));
           ++kit;
           if (n > 0 && !pv(g_it - 1, n == 1)) { fail = true; break; }  // PV(n-1) once its P is stored
           ++g_it;
@@ -1283,8 +1283,10 @@ __device__ __forceinline__ void attn_rows(const AttnParams& p) {
           }
           l_half *= alpha;
           if (n > 0 && __any_sync(kFull, grow)) {
-            // O must hold PV(n-1): S(n) was committed after PV(n-2) only
-            if (__any_sync(kFull, !mbar_wait(b_pv_done, (g_it - 1) & 1, p.wait_limit_ns))) { fail = true; break; }
+            // O must hold PV(n-1): S(n) was committed after PV(n-2) only; PV(n-1) releases V stage
+            // (n-1) % kVStages
+            if (__any_sync(kFull, !mbar_wait(b_v_empty((g_it - 1) % kVStages), ((g_it - 1) / kVStages) & 1,
+                                             p.wait_limit_ns))) { fail = true; break; }
             tc_fence_after();
             const uint64_t a2 = f2_make(alpha, alpha);
 #pragma unroll 1
