@@ -179,7 +179,12 @@ FP_API fp_status fp_block_pool_search(const fp_problem* p, const void* q, const 
  * of local block ids <= i are accepted; out-of-range entries are skipped and flagged).
  * softmax_scale <= 0 selects 1/sqrt(d). out: device bf16 [total_tokens, Hq, d].
  * lse (optional, may be NULL): device float32 [Hq, total_tokens], natural-log sum of
- * exp(softmax_scale * q.k) over the attended keys. */
+ * exp(softmax_scale * q.k) over the attended keys.
+ * For B = 128 two kernels are launched on `stream`, one per attention schedule (two adjacent query
+ * tiles of one head per unit, or one tile per unit); each first sums the list counts, and the one
+ * not chosen returns at once (single tiles when fewer than 40% of the causal blocks are kept). The
+ * choice depends on the lists alone, so a call is deterministic; the two schedules round the
+ * softmax normaliser differently (one bf16 ulp of out at most). */
 FP_API fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,
                                const int32_t* counts, const int32_t* indices, float softmax_scale, void* out,
                                float* lse, int32_t* dev_status, void* stream);
