@@ -183,8 +183,8 @@ FP_API fp_status fp_block_pool_search(const fp_problem* p, const void* q, const 
  * For B = 128 two kernels are launched on `stream`, one per attention schedule (two adjacent query
  * tiles of one head per unit, or one tile per unit); each first sums the list counts, and the one
  * not chosen returns at once (single tiles when fewer than 40% of the causal blocks are kept). The
- * choice depends on the lists alone, so a call is deterministic; the two schedules round the
- * softmax normaliser differently (one bf16 ulp of out at most). */
+ * choice depends on the lists alone, so a call is deterministic; the two schedules add the fp32
+ * softmax terms in different orders, both within the same tolerance of exact attention. */
 FP_API fp_status fp_block_sparse_attn(const fp_problem* p, const void* q, const void* k, const void* v,
                                const int32_t* counts, const int32_t* indices, float softmax_scale, void* out,
                                float* lse, int32_t* dev_status, void* stream);
