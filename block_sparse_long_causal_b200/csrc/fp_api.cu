@@ -180,10 +180,12 @@ fp_status attn_common(const fp_problem* p, const fp_paged_cache* c, const void* 
   // on a barrier that nothing arrives on; the wait runs out, FP_DEV_TIMEOUT is set, the CTA unwinds
   const char* tw = getenv("FP_TEST_UNSIGNALLED_WAIT");
   a.test_unsignalled_wait = (tw && tw[0] == '1') ? 1 : 0;
-  // tuning / test knob: FP_ATTN_UNITS=pairs or rows forces the attention schedule (default: chosen
-  // on the device from the lists' density, for the plain bf16 prefill with B = 128)
+  // tuning / test knob: FP_ATTN_UNITS=pairs or rows forces the attention schedule of the sparse call
+  // (default: chosen on the device from the lists' density, for the plain bf16 prefill with B = 128).
+  // The dense call always runs the paired schedule (the row kernel is not launched for it), so the
+  // knob is not passed on there.
   const char* un = getenv("FP_ATTN_UNITS");
-  a.units = (un && strcmp(un, "pairs") == 0) ? 1 : (un && strcmp(un, "rows") == 0) ? 2 : 0;
+  a.units = dense ? 0 : (un && strcmp(un, "pairs") == 0) ? 1 : (un && strcmp(un, "rows") == 0) ? 2 : 0;
   const int grid = (int)(tiles_ub < sm_count() ? tiles_ub : sm_count());
   return cuda_status(fp::launch_attn(a, grid, static_cast<cudaStream_t>(stream)), "attention launch");
 }
